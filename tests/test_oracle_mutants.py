@@ -1,0 +1,85 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case below plants one mistake in a copy of the oracle's C source (on the
+CPU, in a temporary directory), builds it, binds the oracle module to the
+mutant, and runs the pins of test_oracle_pins.py. At least one pin must fail
+for every mutant; the real oracle is re-bound afterwards.
+"""
+import inspect
+
+import numpy as np
+import pytest
+
+import test_oracle_pins as pins
+
+# (name, text in rq_oracle.c, replacement, occurrence index or None = all)
+MUTANTS = [
+    ("drop the E[x^2] weight", "L = L + ak * e;", "L = L + e;", None),
+    ("ties go to the last index", "L < bestL", "L <= bestL", None),
+    ("qmax = 2^(b-1)", "int qmax = (1 << (bits - 1)) - 1;", "int qmax = (1 << (bits - 1));", None),
+    ("nibbles swapped", "if ((kk & 1) == 0) *byte = u;\n                    else *byte = (uint8_t)(*byte | (u << 4));",
+     "if ((kk & 1) == 1) *byte = u;\n                    else *byte = (uint8_t)(*byte | (u << 4));", None),
+    ("search on the unrounded scale", "float sf = orc_f16_to_f32(sh);\n        double L", "float sf = prod;\n        double L", None),
+    ("truncate instead of rint", "float r = rintf(clampf(v, -(float)qmax, (float)qmax));",
+     "float r = truncf(clampf(v, -(float)qmax, (float)qmax));", None),
+    ("asym offset sign", "float M = (lo_i < 0.0f) ? -lo_i : 0.0f;", "float M = (lo_i < 0.0f) ? lo_i : 0.0f;", None),
+    ("asym step over 16 levels", "float S = (2.0f * r) / 15.0f;", "float S = (2.0f * r) / 16.0f;", None),
+    ("bit string off by one", "int bs = 6 * j + b, bm = 48 + 6 * j + b;", "int bs = 6 * j + b, bm = 47 + 6 * j + b;", None),
+    ("fp16 ties away from zero", "(rem == halfway && (kept & 1u))", "(rem == halfway)", None),
+    ("grid misses its top end", "step = step / (double)(n - 1);", "step = step / (double)n;", None),
+    ("superblock min from the scales", "if (M_star[j] > mM) mM = M_star[j];", "if (S_star[j] > mM) mM = S_star[j];", None),
+    ("product sums the wrong row of x", "const double *xm = xd + (size_t)m * K;", "const double *xm = xd;", None),
+    ("int8 code offset 127", "codes[(size_t)n * K + kk] = (uint8_t)(q[k] + 128);",
+     "codes[(size_t)n * K + kk] = (uint8_t)(q[k] + 127);", None),
+    ("dequant drops the group index", "float s = orc_f16_to_f32(scales[(size_t)n * ng + k / G]);",
+     "float s = orc_f16_to_f32(scales[(size_t)n * ng]);", None),
+    ("sb dequant adds the min", "float p = (float)q * S;\n    return p - M;", "float p = (float)q * S;\n    return p + M;", None),
+    ("absmax from the last element", "if (v > absmax) absmax = v;", "absmax = v;", None),
+]
+
+
+def _pin_calls():
+    """Every pin of test_oracle_pins as a zero-argument callable of orc."""
+    calls = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        params = list(inspect.signature(fn).parameters)
+        marks = getattr(fn, "pytestmark", [])
+        grids = [m.args for m in marks if m.name == "parametrize"]
+        combos = [{}]
+        for argnames, values in grids:
+            names = [a.strip() for a in argnames.split(",")]
+            new = []
+            for c in combos:
+                for v in values:
+                    vv = v if len(names) > 1 else (v,)
+                    new.append({**c, **dict(zip(names, vv))})
+            combos = new
+        for c in combos:
+            if set(params) - {"orc"} <= set(c):
+                calls.append((name, fn, c))
+    return calls
+
+
+@pytest.mark.parametrize("mut", range(len(MUTANTS)), ids=[m[0] for m in MUTANTS])
+def test_a_pin_fails_for_every_planted_mistake(orc, tmp_path, mut):
+    name, old, new, _ = MUTANTS[mut]
+    src = orc.source_text()
+    assert old in src, f"mutation site for '{name}' not found"
+    so = str(tmp_path / "mutant.so")
+    orc.compile_variant(src.replace(old, new), so)
+    prev = orc.swap_library(so)
+    failed = []
+    try:
+        for pname, fn, kw in _pin_calls():
+            try:
+                with np.errstate(all="ignore"):
+                    fn(orc=orc, **kw)
+            except (AssertionError, ValueError, IndexError, OverflowError, ZeroDivisionError):
+                failed.append(pname)
+                break
+    finally:
+        orc.swap_library(None)
+        orc._lib = prev
+    assert failed, f"no pin caught the planted mistake '{name}'"

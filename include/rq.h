@@ -1,0 +1,181 @@
+/*
+ * rq.h -- C ABI of librq: weight-only group-quantized matrix products for
+ * RWKV-7 decode and short prefill on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [ART]  "rwkv-quant: keeping one matrix in bf16 removes 39% of RWKV-7 2.9B's
+ *          quantization loss", section "Two presets and six sizes": the
+ *          REDUCTION preset keeps projections in 8 bits, symmetric, group 16;
+ *          COMPRESSION keeps them in 4 bits with an asymmetric superblock
+ *          layout and group 32; in both, each group's scale and shift are
+ *          found by a search weighted by the input channel's E[x^2].
+ *   [CARD] "RWKV-7 G1 1.5B -- int4 GPTQ for rwkv-sglang", section "Format &
+ *          loading": symmetric int4 weights with group 64, stored as a code
+ *          tensor plus a scale tensor; summary paragraph: the kernels' output
+ *          is bit-identical to the offline dequantization, and an int4 GEMV /
+ *          small-M GEMM / tensor-core GEMM family serves batches up to 32.
+ *
+ * Conventions shared by every call:
+ *   - W is stored [N][K] row-major (row n = output feature, K = input
+ *     features); groups run along K. x is bf16 [M][K], y is fp32 [M][N].
+ *   - Every pointer named "device" is CUDA device memory that the CALLER
+ *     allocated and owns; the library allocates nothing and keeps no state
+ *     between calls. Every such pointer must be 16-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as a
+ *     plain pointer; NULL is the legacy default stream) and never
+ *     synchronizes. Arguments are validated on the host before anything is
+ *     launched; a failed validation launches nothing.
+ *   - A launch that CUDA rejects returns RQ_ERR_CUDA; rq_last_cuda_error()
+ *     then gives the cudaError_t value (per host thread).
+ *   - Non-finite values in W, act_sq or x are outside the contract: the codes
+ *     and outputs they produce are unspecified (but every access stays in
+ *     bounds).
+ *   - Calls made from several host threads on different streams are safe.
+ */
+#ifndef RQ_H
+#define RQ_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rq_status {
+    RQ_OK = 0,
+    RQ_ERR_INVALID_ARG = 1,        /* NULL pointer, M/K/N or search outside range */
+    RQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K not a multiple of the format's block size */
+    RQ_ERR_FORMAT_MISMATCH = 3,    /* descriptor's fmt/K/N differ from the call's */
+    RQ_ERR_MISALIGNED = 4,         /* a device pointer is not 16-byte aligned */
+    RQ_ERR_CUDA = 5,               /* a CUDA runtime call failed */
+    RQ_ERR_DEVICE_TIMEOUT = 6      /* a bounded device wait gave up (see rq_device_status) */
+} rq_status;
+
+/* Packed formats.
+ *
+ * RQ_W4_SYM_G64 ([CARD] "Format & loading"): symmetric int4, group 64.
+ *   codes  [N][K/2] bytes: byte j of row n holds k = 2j in its low nibble
+ *          and k = 2j+1 in its high nibble; nibble = q + 8, q in [-7, 7].
+ *   scales [N][K/64] fp16 (IEEE binary16, little-endian).
+ *   w_hat = q * scale (exact in fp32). 4.25 bits per weight.
+ *
+ * RQ_W8_SYM_G16 ([ART], REDUCTION projections): symmetric int8, group 16.
+ *   codes  [N][K] bytes, byte = q + 128, q in [-127, 127].
+ *   scales [N][K/16] fp16.   w_hat = q * scale. 9 bits per weight.
+ *
+ * RQ_W4_ASYM_SB32 ([ART], COMPRESSION projections): asymmetric int4 in
+ *   superblocks of 256 weights = 8 groups of 32 along K; one 144-byte record
+ *   per superblock, records [N][K/256]:
+ *     [0:2]    fp16 d      superblock scale
+ *     [2:4]    fp16 dmin   superblock min
+ *     [4:16]   96-bit little-endian bit string; bits 6j..6j+5 = sc_j,
+ *              bits 48+6j..48+6j+5 = m_j (6-bit, j = 0..7)
+ *     [16:144] 128 code bytes, nibble order as RQ_W4_SYM_G64, code = q in [0, 15]
+ *   Group j: S_j = d * sc_j, M_j = dmin * m_j; w_hat = S_j * q - M_j
+ *   (S_j * q exact, one fp32 rounding). 4.5 bits per weight; scales = NULL.
+ */
+typedef enum rq_format {
+    RQ_W4_SYM_G64 = 1,
+    RQ_W8_SYM_G16 = 2,
+    RQ_W4_ASYM_SB32 = 3
+} rq_format;
+
+/* Candidate grid of the E[x^2]-weighted search ([ART]): n_cand points
+ * t_i = fp32(t_lo + (t_hi - t_lo) * i / (n_cand - 1)) computed in fp64
+ * (n_cand = 1 gives the single point t_hi). {1, 1.0, 1.0} is plain RTN;
+ * the default (search == NULL) is {64, 0.7, 1.0}.
+ * Limits: 1 <= n_cand <= 256, 0 < t_lo <= t_hi <= 4. */
+typedef struct rq_search {
+    int n_cand;
+    float t_lo;
+    float t_hi;
+} rq_search;
+
+/* Descriptor of one packed matrix. A host struct holding device pointers;
+ * the caller fills it and owns both planes. scales is NULL for
+ * RQ_W4_ASYM_SB32. */
+typedef struct rq_packed {
+    int fmt;        /* rq_format */
+    int K;          /* input features */
+    int N;          /* output features */
+    int reserved;   /* must be 0 */
+    void *codes;    /* device, rq_packed_size(...) codes_bytes */
+    void *scales;   /* device, rq_packed_size(...) scales_bytes, or NULL */
+} rq_packed;
+
+/* Shape limits: 1 <= N <= 2^24; 64 <= K <= 32768 with K % 64 == 0
+ * (K % 256 == 0 for RQ_W4_ASYM_SB32); 1 <= M <= 128. */
+
+/* Bytes of the two planes of a packed [N][K] matrix; the scales plane is
+ * rounded up to a multiple of 16 bytes (the padding is written as zero by
+ * rq_quantize_pack). Returns the total, or 0 for an unknown format or an
+ * unsupported shape. Either out-pointer may be NULL. Host only; no CUDA call. */
+size_t rq_packed_size(int fmt, int K, int N, size_t *codes_bytes, size_t *scales_bytes);
+
+/* Quantize and pack W.  ([ART] "Two presets and six sizes"; [CARD])
+ *   W      device fp32 [N][K]
+ *   act_sq device fp32 [K], E[x_k^2] of the input channels, the weights of
+ *          the search's loss; NULL means every a_k = 1 (plain MSE search).
+ *   search candidate grid; NULL means {64, 0.7, 1.0}.
+ *   out    descriptor whose fmt/K/N must equal the call's and whose planes
+ *          receive the codes and scales.
+ * For each symmetric group: absmax = max|w|, base = absmax / qmax (fp32,
+ * qmax = 7 or 127); candidate i has scale s_i = fp16(t_i * base); its loss is
+ * sum_k a_k (w_k - q_k s_i)^2 with q_k = clamp(rint(w_k / s_i), -qmax, qmax),
+ * evaluated in fp64 in ascending k; the lowest index attaining the minimum
+ * wins. For each asymmetric group of 32: lo = min(0, min w),
+ * hi = max(0, max w), candidate i shrinks [lo, hi] about its midpoint by t_i
+ * (S_i = 2 r_i / 15, M_i = max(0, r_i - mid), r_i = t_i (hi - lo) / 2),
+ * codes q = clamp(rint((w + M_i) / S_i), 0, 15), the same loss and tie rule;
+ * then d = fp16(max_j S_j / 63), dmin = fp16(max_j M_j / 63), 6-bit
+ * sc_j = rint(S_j / d), m_j = rint(M_j / dmin), and the final codes use the
+ * stored S_j = d sc_j, M_j = dmin m_j. The output is byte-for-byte
+ * deterministic. */
+int rq_quantize_pack(const float *W, int K, int N, const float *act_sq,
+                     const rq_search *search, const rq_packed *out, void *stream);
+
+/* y = x * w_hat^T.  ([CARD] summary: an int4 GEMV / small-M GEMM /
+ * tensor-core GEMM family serving batches of 1..32; [ART]: the same product
+ * over the REDUCTION and COMPRESSION projection formats)
+ *   x   device bf16 [M][K] (raw bf16 bit patterns, row-major)
+ *   M   activation rows, 1..128
+ *   K,N must equal the descriptor's
+ *   w   packed matrix
+ *   y   device fp32 [M][N], overwritten (not accumulated into)
+ * w_hat is formed in registers or shared memory and never written out; the
+ * products accumulate in fp32. Kernels are launched with programmatic
+ * dependent launch allowed: they read the packed weights while the kernel
+ * launched just before them on the stream may still be running, and read x
+ * and write y only after it has completed. So the packed planes must not be
+ * written by the kernel launched immediately before rq_wgemm on the same
+ * stream (rq_quantize_pack already ends with a kernel that makes this hold;
+ * after writing the planes with your own kernel, synchronize or launch any
+ * other kernel in between). Copies (cudaMemcpy*) are ordered as usual. */
+int rq_wgemm(const void *x, int M, int K, int N, const rq_packed *w, float *y, void *stream);
+
+/* Export w_hat as fp32 [N][K] into W_out (device).  ([CARD] summary: the
+ * kernel output is bit-identical to the offline dequantization.) Uses the
+ * same device unpack as rq_wgemm; bit-exact: q * scale for the symmetric
+ * formats, fp32(S_j * q - M_j) for the superblock format. */
+int rq_dequant(const rq_packed *w, float *W_out, void *stream);
+
+/* Static description of a status code. Never NULL. */
+const char *rq_status_string(int status);
+
+/* cudaError_t of the last RQ_ERR_CUDA returned on this host thread (0 if none). */
+int rq_last_cuda_error(void);
+
+/* Reads and clears the device status word that bounded waits inside the
+ * tensor-core kernels set when they give up. Synchronizes `stream`.
+ * Writes the word to *word (0 = no timeout since the last read) and returns
+ * RQ_OK, RQ_ERR_DEVICE_TIMEOUT if the word was non-zero, or RQ_ERR_CUDA. */
+int rq_device_status(void *stream, int *word);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int rq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQ_H */

@@ -1,0 +1,206 @@
+"""Python binding of librq (include/rq.h): weight-only group-quantized matrix
+products for RWKV-7 on B200.
+
+This module only marshals arguments: it passes torch tensors' device pointers
+and the current CUDA stream to the C ABI. PyTorch provides device memory and
+streams; every step of the computation runs in librq's CUDA kernels. There is
+no fallback: if librq.so is missing, every call raises.
+
+Formats (see include/rq.h): ``RQ_W4_SYM_G64`` (symmetric int4, group 64),
+``RQ_W8_SYM_G16`` (symmetric int8, group 16), ``RQ_W4_ASYM_SB32`` (asymmetric
+int4 superblocks of 8 groups of 32). The strings "w4g64", "w8g16", "w4sb32"
+are accepted wherever a format is expected.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librq.so")
+
+RQ_OK = 0
+RQ_ERR_INVALID_ARG = 1
+RQ_ERR_UNSUPPORTED_SHAPE = 2
+RQ_ERR_FORMAT_MISMATCH = 3
+RQ_ERR_MISALIGNED = 4
+RQ_ERR_CUDA = 5
+RQ_ERR_DEVICE_TIMEOUT = 6
+
+RQ_W4_SYM_G64 = 1
+RQ_W8_SYM_G16 = 2
+RQ_W4_ASYM_SB32 = 3
+FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_ASYM_SB32}
+EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_dequant", "rq_status_string",
+           "rq_last_cuda_error", "rq_device_status", "rq_version")
+
+
+class RqSearch(ctypes.Structure):
+    _fields_ = [("n_cand", ctypes.c_int), ("t_lo", ctypes.c_float), ("t_hi", ctypes.c_float)]
+
+
+class RqPacked(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int), ("K", ctypes.c_int), ("N", ctypes.c_int), ("reserved", ctypes.c_int),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class RqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {rq_status_string(status)} (status {status})"
+        if status == RQ_ERR_CUDA:
+            msg += f", cudaError {_lib().rq_last_cuda_error()}"
+        super().__init__(msg)
+
+
+_L = None
+
+
+def _lib() -> ctypes.CDLL:
+    """Load librq.so (built in-tree). Raises if it is absent: there is no
+    other implementation to fall back to."""
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"librq.so is not built ({LIB_PATH}); run "
+                              "`python -m weight_only_quantized_rq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.rq_packed_size.argtypes = [I, I, I, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+        L.rq_packed_size.restype = ctypes.c_size_t
+        L.rq_quantize_pack.argtypes = [P, I, I, P, ctypes.POINTER(RqSearch), ctypes.POINTER(RqPacked), P]
+        L.rq_quantize_pack.restype = I
+        L.rq_wgemm.argtypes = [P, I, I, I, ctypes.POINTER(RqPacked), P, P]
+        L.rq_wgemm.restype = I
+        L.rq_dequant.argtypes = [ctypes.POINTER(RqPacked), P, P]
+        L.rq_dequant.restype = I
+        L.rq_status_string.argtypes = [I]
+        L.rq_status_string.restype = ctypes.c_char_p
+        L.rq_last_cuda_error.argtypes = []
+        L.rq_last_cuda_error.restype = I
+        L.rq_device_status.argtypes = [P, ctypes.POINTER(I)]
+        L.rq_device_status.restype = I
+        L.rq_version.argtypes = []
+        L.rq_version.restype = I
+        _L = L
+    return _L
+
+
+def lib() -> ctypes.CDLL:
+    return _lib()
+
+
+def fmt_id(fmt) -> int:
+    return FORMAT_IDS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _check(status: int, where: str) -> None:
+    if status != RQ_OK:
+        raise RqError(status, where)
+
+
+# ------------------------------------------------------------------ calls --
+def rq_status_string(status: int) -> str:
+    return _lib().rq_status_string(int(status)).decode()
+
+
+def rq_version() -> int:
+    return _lib().rq_version()
+
+
+def rq_packed_size(fmt, K: int, N: int) -> tuple[int, int]:
+    """(codes_bytes, scales_bytes); raises for an unsupported shape."""
+    cb, sb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    tot = _lib().rq_packed_size(fmt_id(fmt), int(K), int(N), ctypes.byref(cb), ctypes.byref(sb))
+    if tot == 0:
+        raise RqError(RQ_ERR_UNSUPPORTED_SHAPE, "rq_packed_size")
+    return cb.value, sb.value
+
+
+@dataclass
+class Packed:
+    """A packed matrix: the descriptor fields plus the two device planes
+    (uint8 tensors that own the memory)."""
+    fmt: int
+    K: int
+    N: int
+    codes: torch.Tensor
+    scales: torch.Tensor | None
+
+    def desc(self) -> RqPacked:
+        return RqPacked(self.fmt, self.K, self.N, 0, self.codes.data_ptr(),
+                        None if self.scales is None else self.scales.data_ptr())
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() + (0 if self.scales is None else self.scales.numel())
+
+
+def alloc_packed(fmt, K: int, N: int, device=None) -> Packed:
+    f = fmt_id(fmt)
+    cb, sb = rq_packed_size(f, K, N)
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    codes = torch.empty(cb, dtype=torch.uint8, device=dev)
+    scales = torch.empty(sb, dtype=torch.uint8, device=dev) if sb else None
+    return Packed(f, int(K), int(N), codes, scales)
+
+
+def rq_quantize_pack(W: torch.Tensor, fmt, act_sq: torch.Tensor | None = None, n_cand: int = 64,
+                     t_lo: float = 0.7, t_hi: float = 1.0, out: Packed | None = None, stream=None) -> Packed:
+    """Quantize and pack W (fp32 [N][K], CUDA). Returns the Packed matrix."""
+    N, K = W.shape
+    if out is None:
+        out = alloc_packed(fmt, K, N, W.device)
+    sr = RqSearch(int(n_cand), float(t_lo), float(t_hi))
+    d = out.desc()
+    _check(_lib().rq_quantize_pack(_ptr(W), int(K), int(N), _ptr(act_sq), ctypes.byref(sr), ctypes.byref(d),
+                                   _stream(stream)), "rq_quantize_pack")
+    return out
+
+
+def rq_wgemm(x: torch.Tensor, w: Packed, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x @ w_hat.T with x bf16 [M][K] and y fp32 [M][N] (CUDA tensors)."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty(M, w.N, dtype=torch.float32, device=x.device)
+    d = w.desc()
+    _check(_lib().rq_wgemm(_ptr(x), int(M), int(K), int(w.N), ctypes.byref(d), _ptr(y), _stream(stream)),
+           "rq_wgemm")
+    return y
+
+
+def rq_dequant(w: Packed, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """w_hat as fp32 [N][K] (CUDA)."""
+    if out is None:
+        out = torch.empty(w.N, w.K, dtype=torch.float32, device=w.codes.device)
+    d = w.desc()
+    _check(_lib().rq_dequant(ctypes.byref(d), _ptr(out), _stream(stream)), "rq_dequant")
+    return out
+
+
+def rq_device_status(stream=None) -> int:
+    """Read and clear the device status word (synchronizes the stream)."""
+    word = ctypes.c_int(0)
+    st = _lib().rq_device_status(_stream(stream), ctypes.byref(word))
+    if st not in (RQ_OK, RQ_ERR_DEVICE_TIMEOUT):
+        raise RqError(st, "rq_device_status")
+    return word.value
+
+
+# short aliases
+quantize_pack = rq_quantize_pack
+wgemm = rq_wgemm
+dequant = rq_dequant
+packed_size = rq_packed_size

@@ -1,0 +1,183 @@
+// rq_device.cuh -- device-side building blocks shared by librq's kernels:
+// inline-PTX wrappers (mbarrier, bulk async copy, programmatic dependent
+// launch), bounded waits, and the in-register unpack of packed codes.
+//
+// The unpack functions are the single definition of how a stored code becomes
+// a number; rq_dequant and the GEMV both use them, so the exported w_hat and
+// the w_hat inside the product are the same values ("kernel output is
+// bit-identical to the offline dequant": RWKV-7 G1 1.5B int4 model card,
+// summary paragraph).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+namespace rq {
+
+// ---------------------------------------------------------------- status ---
+// Bit flags of the device status word (one per device, read and cleared by
+// rq_device_status). A bounded wait that gives up ORs its bit in and returns.
+enum : unsigned {
+    kStatusTmaWait = 1u << 0,    // waited too long for an async copy
+    kStatusSlotWait = 1u << 1,   // waited too long for a ring slot to free
+    kStatusMmaWait = 1u << 2,    // waited too long for a tensor-core commit
+    kStatusTmem = 1u << 3,       // TMEM allocation did not succeed
+};
+
+// One word per translation unit (internal linkage, so no device linking is
+// needed); each kernel file exports a host accessor that reads and clears it.
+static __device__ unsigned g_status = 0u;
+
+// Wall-clock bound of every device spin-wait, in nanoseconds.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// -------------------------------------------------------------- mbarrier ---
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete. Gives up after
+// kWaitLimitNs, ORs `flag` into the device status word and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, flag);
+            return false;
+        }
+    }
+}
+
+// ------------------------------------------------------ bulk async copy ---
+// One contiguous global -> shared copy completed on an mbarrier (the untiled
+// TMA form). dst, src and bytes must be multiples of 16. Loads with an L2
+// evict-first policy: the packed weights are streamed once per call.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// -------------------------------------------- programmatic dependent launch
+// The packed weights never depend on the previous kernel, so kernels prefetch
+// them before grid_dep_wait(); x and y are touched only after it.
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------- loads ------
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+    return v;
+}
+__device__ __forceinline__ float4 lds128f(const void* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(smem_u32(p)));
+    return v;
+}
+
+// --------------------------------------------------------------- unpack ---
+// int4 codes. A 32-bit word holds eight nibbles; nibble p (bits 4p..4p+3)
+// is the code of weight k = 8i + p of that word (byte j: k = 2j low, 2j+1
+// high). unpack_w4 turns the word into eight fp32 values 128 + u exactly:
+// each nibble is placed in bits 16..19 under the exponent byte 0x43 (fp32
+// 128.0, whose mantissa bit 16 weighs 1), one byte permute per value.
+// Output order: f[0..3] = nibbles 0, 2, 4, 6 (low nibble of bytes 0..3),
+//               f[4..7] = nibbles 1, 3, 5, 7 (high nibble of bytes 0..3).
+constexpr uint32_t kW4Magic = 0x43000000u;  // 128.0f
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ void unpack_w4(uint32_t w, float f[8]) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
+    // prmt selector nibbles pick bytes of {b = magic (bytes 4..7), a (bytes 0..3)}:
+    // result byte3 = 0x43 (selector 7), byte2 = a.byte_k, bytes1..0 = 0x00 (selector 4)
+    f[0] = __uint_as_float(prmt(lo, kW4Magic, 0x7044u));
+    f[1] = __uint_as_float(prmt(lo, kW4Magic, 0x7144u));
+    f[2] = __uint_as_float(prmt(lo, kW4Magic, 0x7244u));
+    f[3] = __uint_as_float(prmt(lo, kW4Magic, 0x7344u));
+    f[4] = __uint_as_float(prmt(hi, kW4Magic, 0x7044u));
+    f[5] = __uint_as_float(prmt(hi, kW4Magic, 0x7144u));
+    f[6] = __uint_as_float(prmt(hi, kW4Magic, 0x7244u));
+    f[7] = __uint_as_float(prmt(hi, kW4Magic, 0x7344u));
+}
+// Position inside the word of output slot j of unpack_w4.
+__host__ __device__ constexpr int w4_slot_nibble(int j) { return j < 4 ? 2 * j : 2 * (j - 4) + 1; }
+
+// int8 codes. Byte k of a word is the code u = q + 128 of weight k. Each byte
+// is placed in bits 8..15 under exponent byte 0x47 (fp32 32768.0, mantissa
+// bit 8 weighs 1), giving 32768 + u; subtracting 32896 gives q exactly.
+constexpr uint32_t kW8Magic = 0x47000000u;  // 32768.0f
+
+__device__ __forceinline__ void unpack_w8(uint32_t w, float f[4]) {
+    f[0] = __fsub_rn(__uint_as_float(prmt(w, kW8Magic, 0x7404u)), 32896.0f);
+    f[1] = __fsub_rn(__uint_as_float(prmt(w, kW8Magic, 0x7414u)), 32896.0f);
+    f[2] = __fsub_rn(__uint_as_float(prmt(w, kW8Magic, 0x7424u)), 32896.0f);
+    f[3] = __fsub_rn(__uint_as_float(prmt(w, kW8Magic, 0x7434u)), 32896.0f);
+}
+
+// Superblock header: 6-bit field of group j (which = 0: scale, 1: min) from
+// the 96-bit string held in words b0 (bits 0..31), b1 (32..63), b2 (64..95).
+__device__ __forceinline__ uint32_t sb_field(uint32_t b0, uint32_t b1, uint32_t b2, int which, int j) {
+    const int s = 48 * which + 6 * j;
+    const uint32_t lo = s < 32 ? b0 : (s < 64 ? b1 : b2);
+    const uint32_t hi = s < 32 ? b1 : (s < 64 ? b2 : 0u);
+    return __funnelshift_r(lo, hi, s & 31) & 63u;
+}
+
+}  // namespace rq

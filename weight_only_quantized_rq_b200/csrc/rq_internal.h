@@ -1,0 +1,57 @@
+// rq_internal.h -- host-side interfaces between librq's C ABI layer
+// (rq_api.cu) and its kernel files. Not installed; not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace rq {
+
+constexpr int kFmtW4G64 = 1;
+constexpr int kFmtW8G16 = 2;
+constexpr int kFmtW4SB32 = 3;
+
+// Bytes per row of the codes plane (records plane for the superblock format)
+// and of the scales plane.
+inline size_t code_row_bytes(int fmt, int K) {
+    return fmt == kFmtW4G64 ? (size_t)K / 2 : fmt == kFmtW8G16 ? (size_t)K : (size_t)K / 256 * 144;
+}
+inline size_t scale_row_bytes(int fmt, int K) {
+    return fmt == kFmtW4G64 ? (size_t)K / 32 : fmt == kFmtW8G16 ? (size_t)K / 8 : 0;
+}
+inline size_t round16(size_t v) { return (v + 15) & ~(size_t)15; }
+
+struct PackArgs {
+    int fmt, K, N;
+    const float* W;
+    const float* act_sq;
+    int n_cand;
+    float t_lo, t_hi;
+    void* codes;
+    void* scales;
+    size_t scales_bytes;   // padded plane size (padding is zeroed)
+};
+
+cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st);
+cudaError_t launch_dequant(int fmt, int K, int N, const void* codes, const void* scales, float* out,
+                           cudaStream_t st);
+
+struct WgemmArgs {
+    int fmt, M, K, N;
+    const void* x;         // bf16 [M][K]
+    const void* codes;
+    const void* scales;
+    float* y;              // fp32 [M][N]
+};
+
+// Memory-bound path (few activation rows): dequantize in registers, fp32 FMA.
+cudaError_t launch_gemv(const WgemmArgs& a, cudaStream_t st);
+
+// Read and clear the device status word of each kernel file (synchronizes st).
+cudaError_t status_pack(cudaStream_t st, unsigned* word);
+cudaError_t status_gemv(cudaStream_t st, unsigned* word);
+
+int sm_count();   // multiprocessors of the current device
+
+}  // namespace rq

@@ -1,0 +1,375 @@
+// rq_pack.cu -- quantize-pack (RTN / E[x^2]-weighted grid search) and the
+// dequant export, for the three packed formats.
+//
+// Sources: rwkv-quant article ("rwkv-quant: keeping one matrix in bf16 removes
+// 39% of RWKV-7 2.9B's quantization loss", section "Two presets and six
+// sizes"): symmetric int8 group 16 (REDUCTION), asymmetric int4 superblock
+// group 32 (COMPRESSION), each group's scale and shift found by a search
+// weighted by E[x^2] of the input channel. RWKV-7 G1 1.5B int4 model card
+// ("Format & loading"): symmetric int4 group 64 as codes plus scales.
+//
+// Determinism: every fp32 / fp64 operation on the search path is an explicit
+// round-to-nearest intrinsic (never contracted into an FMA), each candidate's
+// loss is summed sequentially in ascending k by one thread, and the argmin
+// keeps the lowest index among equal losses. The output bytes therefore do
+// not depend on the launch shape.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "rq_device.cuh"
+#include "rq_internal.h"
+
+namespace rq {
+namespace {
+
+// Candidate t_i = fp32(lo + (hi - lo) * i / (n - 1)) in fp64; n = 1 -> hi.
+__device__ __forceinline__ float cand_t(int i, int n, float t_lo, float t_hi) {
+    if (n == 1) return t_hi;
+    const double lo = (double)t_lo, hi = (double)t_hi;
+    double step = __dmul_rn(__dsub_rn(hi, lo), (double)i);
+    step = __ddiv_rn(step, (double)(n - 1));
+    return __double2float_rn(__dadd_rn(lo, step));
+}
+
+__device__ __forceinline__ float clampf(float v, float lo, float hi) {
+    return v < lo ? lo : (v > hi ? hi : v);
+}
+
+// Symmetric code for scale sf: clamp(rint(w / sf), -qmax, qmax); 0 if sf == 0.
+__device__ __forceinline__ int sym_code(float w, float sf, float qmax) {
+    if (sf == 0.0f) return 0;
+    return (int)rintf(clampf(__fdiv_rn(w, sf), -qmax, qmax));
+}
+
+// Asymmetric code: clamp(rint((w + M) / S), 0, 15); 0 if S == 0.
+__device__ __forceinline__ int asym_code(float w, float S, float M) {
+    if (S == 0.0f) return 0;
+    return (int)rintf(clampf(__fdiv_rn(__fadd_rn(w, M), S), 0.0f, 15.0f));
+}
+
+// (loss, index) pair reduction over a warp: smallest loss, then smallest index.
+__device__ __forceinline__ void warp_argmin(double& L, int& idx) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double L2 = __shfl_xor_sync(0xffffffffu, L, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+        if (L2 < L || (L2 == L && i2 < idx)) { L = L2; idx = i2; }
+    }
+}
+
+constexpr int kPackWarps = 8;
+constexpr double kInf = __builtin_huge_val();
+
+// One warp per symmetric group of G weights (G = 64: int4, qmax 7;
+// G = 16: int8, qmax 127). Lane l evaluates candidates l, l+32, ...
+template <int G, int QMAX>
+__global__ void __launch_bounds__(kPackWarps * 32)
+qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
+                 int n_cand, float t_lo, float t_hi, uint8_t* __restrict__ codes,
+                 uint16_t* __restrict__ scales) {
+    __shared__ float s_w[kPackWarps][G];
+    __shared__ float s_a[kPackWarps][G];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ng = K / G;
+    const long long total = (long long)N * ng;
+    const long long gid = (long long)blockIdx.x * kPackWarps + warp;
+    if (gid >= total) return;
+    const int n = (int)(gid / ng), g = (int)(gid % ng);
+    const float* w = W + (size_t)n * K + (size_t)g * G;
+
+    float amax = 0.0f;
+    for (int k = lane; k < G; k += 32) {
+        const float v = w[k];
+        s_w[warp][k] = v;
+        s_a[warp][k] = act_sq ? act_sq[(size_t)g * G + k] : 1.0f;
+        amax = fmaxf(amax, fabsf(v));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    __syncwarp();
+    const float qmax = (float)QMAX;
+    const float base = __fdiv_rn(amax, qmax);
+
+    __half best_s;
+    if (n_cand == 1) {
+        best_s = __float2half_rn(__fmul_rn(cand_t(0, 1, t_lo, t_hi), base));
+    } else {
+        double bestL = kInf;   // lanes without a candidate never win
+        int bestI = 0x7fffffff;
+        for (int i = lane; i < n_cand; i += 32) {
+            const float sf = __half2float(__float2half_rn(__fmul_rn(cand_t(i, n_cand, t_lo, t_hi), base)));
+            double L = 0.0;
+            for (int k = 0; k < G; ++k) {
+                const float wk = s_w[warp][k];
+                const float wq = __fmul_rn((float)sym_code(wk, sf, qmax), sf);
+                const double d = __dsub_rn((double)wk, (double)wq);
+                L = __dadd_rn(L, __dmul_rn((double)s_a[warp][k], __dmul_rn(d, d)));
+            }
+            if (bestI == 0x7fffffff || L < bestL) { bestL = L; bestI = i; }
+        }
+        warp_argmin(bestL, bestI);
+        best_s = __float2half_rn(__fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), base));
+    }
+    const float sf = __half2float(best_s);
+    if (G == 64) {
+        // lane l writes byte l of the group: k = 2l (low nibble), 2l+1 (high)
+        const int q0 = sym_code(s_w[warp][2 * lane], sf, qmax);
+        const int q1 = sym_code(s_w[warp][2 * lane + 1], sf, qmax);
+        codes[(size_t)n * (K / 2) + (size_t)g * 32 + lane] = (uint8_t)((q0 + 8) | ((q1 + 8) << 4));
+    } else {
+        if (lane < G) {
+            const int q = sym_code(s_w[warp][lane], sf, qmax);
+            codes[(size_t)n * K + (size_t)g * G + lane] = (uint8_t)(q + 128);
+        }
+    }
+    if (lane == 0) scales[(size_t)n * ng + g] = __half_as_ushort(best_s);
+}
+
+// One block per superblock of 256 weights: warp j searches group j (32
+// weights), then the block forms d, dmin, the 6-bit fields and the codes.
+__global__ void __launch_bounds__(256)
+qpack_sb32_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
+                  int n_cand, float t_lo, float t_hi, uint8_t* __restrict__ blocks) {
+    __shared__ float s_w[256];
+    __shared__ float s_a[256];
+    __shared__ float s_S[8], s_M[8];     // searched S*_j, M*_j
+    __shared__ float s_Sq[8], s_Mq[8];   // stored S_j = d sc_j, M_j = dmin m_j
+    __shared__ __align__(16) uint8_t s_blk[144];
+    const int nb = K / 256;
+    const long long sb = blockIdx.x;
+    const int n = (int)(sb / nb), b = (int)(sb % nb);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const size_t k0 = (size_t)b * 256;
+    s_w[t] = W[(size_t)n * K + k0 + t];
+    s_a[t] = act_sq ? act_sq[k0 + t] : 1.0f;
+    __syncthreads();
+
+    {   // group search (warp = group j)
+        const float* w = s_w + 32 * warp;
+        const float* a = s_a + 32 * warp;
+        float lo = w[lane] < 0.0f ? w[lane] : 0.0f;
+        float hi = w[lane] > 0.0f ? w[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+            const float h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+            lo = l2 < lo ? l2 : lo;
+            hi = h2 > hi ? h2 : hi;
+        }
+        const float half = __fmul_rn(__fsub_rn(hi, lo), 0.5f);
+        const float mid = __fmul_rn(__fadd_rn(hi, lo), 0.5f);
+        double bestL = kInf;
+        int bestI = 0x7fffffff;
+        for (int i = lane; i < n_cand; i += 32) {
+            const float r = __fmul_rn(cand_t(i, n_cand, t_lo, t_hi), half);
+            const float S = __fdiv_rn(__fmul_rn(2.0f, r), 15.0f);
+            const float loi = __fsub_rn(mid, r);
+            const float M = loi < 0.0f ? -loi : 0.0f;
+            double L = 0.0;
+            if (n_cand > 1) {
+                for (int k = 0; k < 32; ++k) {
+                    const float wk = w[k];
+                    const float wq = __fsub_rn(__fmul_rn((float)asym_code(wk, S, M), S), M);
+                    const double d = __dsub_rn((double)wk, (double)wq);
+                    L = __dadd_rn(L, __dmul_rn((double)a[k], __dmul_rn(d, d)));
+                }
+            }
+            if (bestI == 0x7fffffff || L < bestL) { bestL = L; bestI = i; }
+        }
+        warp_argmin(bestL, bestI);
+        if (lane == 0) {
+            const float r = __fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), half);
+            const float loi = __fsub_rn(mid, r);
+            s_S[warp] = __fdiv_rn(__fmul_rn(2.0f, r), 15.0f);
+            s_M[warp] = loi < 0.0f ? -loi : 0.0f;
+        }
+    }
+    __syncthreads();
+
+    if (warp == 0) {   // superblock scale/min and the 6-bit fields
+        float mS = 0.0f, mM = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            mS = s_S[j] > mS ? s_S[j] : mS;
+            mM = s_M[j] > mM ? s_M[j] : mM;
+        }
+        const __half dh = __float2half_rn(__fdiv_rn(mS, 63.0f));
+        const __half mh = __float2half_rn(__fdiv_rn(mM, 63.0f));
+        const float d = __half2float(dh), dm = __half2float(mh);
+        uint32_t field = 0;   // lanes 0..7: sc_j, lanes 8..15: m_j
+        if (lane < 16) {
+            const int j = lane & 7;
+            const float num = lane < 8 ? s_S[j] : s_M[j];
+            const float den = lane < 8 ? d : dm;
+            field = den == 0.0f ? 0u : (uint32_t)(int)rintf(clampf(__fdiv_rn(num, den), 0.0f, 63.0f));
+            if (lane < 8) s_Sq[j] = __fmul_rn(d, (float)field);
+            else s_Mq[j] = __fmul_rn(dm, (float)field);
+        }
+        // assemble the 96-bit string: field f (0..15) at bit 6f
+        uint32_t words[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int f = 0; f < 16; ++f) {
+            const uint64_t v = (uint64_t)__shfl_sync(0xffffffffu, field, f);
+            const int bit = 6 * f;
+            const int wi = bit >> 5, sh = bit & 31;
+            const uint64_t placed = v << sh;
+            words[wi] |= (uint32_t)placed;
+            if (wi + 1 < 3) words[wi + 1] |= (uint32_t)(placed >> 32);
+        }
+        if (lane == 0) {
+            uint32_t* hdr = reinterpret_cast<uint32_t*>(s_blk);
+            hdr[0] = (uint32_t)__half_as_ushort(dh) | ((uint32_t)__half_as_ushort(mh) << 16);
+            hdr[1] = words[0];
+            hdr[2] = words[1];
+            hdr[3] = words[2];
+        }
+    }
+    __syncthreads();
+    if (t < 128) {   // code byte t: k = 2t (low nibble), 2t+1 (high)
+        const int j = (2 * t) >> 5;
+        const float S = s_Sq[j], M = s_Mq[j];
+        const int q0 = asym_code(s_w[2 * t], S, M);
+        const int q1 = asym_code(s_w[2 * t + 1], S, M);
+        s_blk[16 + t] = (uint8_t)(q0 | (q1 << 4));
+    }
+    __syncthreads();
+    if (t < 9) {
+        uint4* dst = reinterpret_cast<uint4*>(blocks + ((size_t)n * nb + b) * 144);
+        dst[t] = reinterpret_cast<const uint4*>(s_blk)[t];
+    }
+}
+
+__global__ void zero_bytes_kernel(uint8_t* p, int n) {
+    if ((int)threadIdx.x < n) p[threadIdx.x] = 0;
+}
+
+// An empty kernel launched with ordinary stream ordering after the packing
+// kernels. rq_wgemm's kernels may start (and read the packed planes) while the
+// kernel launched just before them is still running; putting this one in
+// between guarantees that the packing grid has completed first.
+__global__ void pack_done_kernel() {}
+
+// ---------------------------------------------------------------- dequant --
+// One thread per 32-bit word of codes; writes fp32 w_hat in natural k order.
+__global__ void dequant_w4_kernel(const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
+                                  int K, long long words, float* __restrict__ out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= words) return;
+    const long long wpr = K / 8;
+    const long long n = i / wpr;
+    const int k0 = (int)(i % wpr) * 8;
+    const float s = __half2float(scales[n * (K / 64) + k0 / 64]);
+    float f[8], o[8];
+    unpack_w4(codes[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[w4_slot_nibble(j)] = __fmul_rn(__fsub_rn(f[j], 136.0f), s);
+    float4* dst = reinterpret_cast<float4*>(out + n * K + k0);
+    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+__global__ void dequant_w8_kernel(const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
+                                  int K, long long words, float* __restrict__ out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= words) return;
+    const long long wpr = K / 4;
+    const long long n = i / wpr;
+    const int k0 = (int)(i % wpr) * 4;
+    const float s = __half2float(scales[n * (K / 16) + k0 / 16]);
+    float f[4];
+    unpack_w8(codes[i], f);
+    *reinterpret_cast<float4*>(out + n * K + k0) =
+        make_float4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
+}
+
+// One thread per 32-bit word of a superblock's codes (32 words per record).
+__global__ void dequant_sb32_kernel(const uint8_t* __restrict__ blocks, int K, long long words,
+                                    float* __restrict__ out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= words) return;
+    const long long rec = i / 32;
+    const int wi = (int)(i % 32);
+    const int nb = K / 256;
+    const long long n = rec / nb;
+    const int b = (int)(rec % nb);
+    const uint32_t* r = reinterpret_cast<const uint32_t*>(blocks + rec * 144);
+    const uint32_t h0 = r[0];
+    const float d = __half2float(__ushort_as_half((unsigned short)(h0 & 0xffffu)));
+    const float dm = __half2float(__ushort_as_half((unsigned short)(h0 >> 16)));
+    const int j = wi / 4;   // 4 words (32 weights) per group
+    const float S = __fmul_rn(d, (float)sb_field(r[1], r[2], r[3], 0, j));
+    const float M = __fmul_rn(dm, (float)sb_field(r[1], r[2], r[3], 1, j));
+    float f[8], o[8];
+    unpack_w4(r[4 + wi], f);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) o[w4_slot_nibble(s)] = __fmaf_rn(S, __fsub_rn(f[s], 128.0f), -M);
+    float4* dst = reinterpret_cast<float4*>(out + n * K + (size_t)b * 256 + wi * 8);
+    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st) {
+    const long long N = a.N;
+    if (a.fmt == kFmtW4SB32) {
+        const long long blocksN = N * (a.K / 256);
+        qpack_sb32_kernel<<<(unsigned)blocksN, 256, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo, a.t_hi,
+                                                              static_cast<uint8_t*>(a.codes));
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        pack_done_kernel<<<1, 32, 0, st>>>();
+        return cudaGetLastError();
+    }
+    const int G = a.fmt == kFmtW4G64 ? 64 : 16;
+    const long long groups = N * (a.K / G);
+    const unsigned grid = (unsigned)((groups + kPackWarps - 1) / kPackWarps);
+    if (a.fmt == kFmtW4G64)
+        qpack_sym_kernel<64, 7><<<grid, kPackWarps * 32, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo,
+                                                                   a.t_hi, static_cast<uint8_t*>(a.codes),
+                                                                   static_cast<uint16_t*>(a.scales));
+    else
+        qpack_sym_kernel<16, 127><<<grid, kPackWarps * 32, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo,
+                                                                     a.t_hi, static_cast<uint8_t*>(a.codes),
+                                                                     static_cast<uint16_t*>(a.scales));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t used = (size_t)groups * 2;
+    if (a.scales_bytes > used) {
+        zero_bytes_kernel<<<1, 32, 0, st>>>(static_cast<uint8_t*>(a.scales) + used, (int)(a.scales_bytes - used));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    pack_done_kernel<<<1, 32, 0, st>>>();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(int fmt, int K, int N, const void* codes, const void* scales, float* out,
+                           cudaStream_t st) {
+    const int threads = 256;
+    if (fmt == kFmtW4G64) {
+        const long long words = (long long)N * K / 8;
+        dequant_w4_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
+            static_cast<const uint32_t*>(codes), static_cast<const __half*>(scales), K, words, out);
+    } else if (fmt == kFmtW8G16) {
+        const long long words = (long long)N * K / 4;
+        dequant_w8_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
+            static_cast<const uint32_t*>(codes), static_cast<const __half*>(scales), K, words, out);
+    } else {
+        const long long words = (long long)N * (K / 256) * 32;
+        dequant_sb32_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
+            static_cast<const uint8_t*>(codes), K, words, out);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t status_pack(cudaStream_t st, unsigned* word) {
+    unsigned v = 0, z = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(v), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_status, &z, sizeof(z), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    *word = v;
+    return e;
+}
+
+}  // namespace rq

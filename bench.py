@@ -1,0 +1,378 @@
+"""Benchmark of the decode hot path: the int4 group-64 (E[x^2]-searched)
+weight-only product over the RWKV-7 1.5B layer set, 24 layers x (r, k, v, o
+2048x2048, channel-mix key 2048->8192, value 8192->2048), M = 1 activation
+row, on one B200 per process.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload IDX] [--M ROWS] [--no-graph]
+
+A step is one pass of rq_wgemm over all 144 matrices (the packing is done
+once, before timing; it is offline work in the method). The metric is the
+effective weight-stream bandwidth: packed bytes of all matrices / step time.
+Inputs are synthetic (seeded), weights drawn on the GPU; the packed set
+(642 MB) is larger than the 126 MB L2, so no flush is needed between steps.
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(independent replicas, no collective in the data path: weak scaling); rank 0
+prints the aggregate. ``--impl reference`` times the CPU oracle instead, on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4g64 GEMV effective weight GB/s and % of HBM peak at M=1 (1×B200)"
+HBM_FALLBACK = 6650.0
+NOMINAL_HBM = 8000.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return HBM_FALLBACK, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------- clocks -------
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"rq_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ oracle ------
+def oracle_sample(w, seconds: float, seed: int = 0):
+    """Time the CPU oracle's product (exact dequant + fp64 sums) over a
+    bounded sample of the workload's rows: for each matrix shape of one
+    layer, a few rows (packed by the oracle from CPU-drawn weights). Returns
+    (packed bytes processed per second, description, threads)."""
+    import numpy as np
+
+    import oracle
+    from weight_only_quantized_rq_b200 import workloads as wl
+    oracle.build()
+    rng = np.random.default_rng(seed)
+    shapes = []
+    for j, layer, m in w.matrices():
+        if layer > 0:
+            break
+        rows = 128
+        g = wl.random_matrix(10_000 + j, rows, m.K).numpy()
+        a = wl.act_sq(w, m.K)
+        codes, scales = oracle.pack(m.fmt, g, a if m.n_cand > 1 else None, n_cand=m.n_cand,
+                                    t_lo=0.7 if m.n_cand > 1 else 1.0)
+        x = wl.bf16_bits(wl.activations(w, j, m.K, 1))
+        import weight_only_quantized_rq_b200 as rq_
+        cb, sb = rq_.rq_packed_size(m.fmt, m.K, m.N)
+        per_row = (cb + sb) / m.N
+        shapes.append((m, codes, scales, x, rows, per_row))
+    done_bytes, t0 = 0.0, time.perf_counter()
+    reps = 0
+    while True:
+        for m, codes, scales, x, rows, per_row in shapes:
+            oracle.wgemm(m.fmt, x, m.K, rows, codes, scales)
+            done_bytes += rows * per_row
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    desc = (f"oracle product (exact dequant + fp64 ascending-k sums) over 128 rows of each of the "
+            f"{len(shapes)} matrix shapes of one layer, M=1, repeated {reps}x ({el:.1f} s)")
+    return done_bytes / el / 1e9, desc, oracle.threads(), el
+
+
+def run_reference(args, w, M):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    per_step = 2.0
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step / 4)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, desc, thr, el = oracle_sample(w, per_step)
+        vals.append(v)
+        secs.append(el)
+    value = statistics.median(vals)
+    hbm, src = peaks()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.median(secs), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, M),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": thr, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, M):
+    return {"workload": w.name, "M": M, "matrices": len(w.matrices()),
+            "formats": sorted({m.fmt for m in w.per_layer}),
+            "l2": "packed set larger than the 126 MB L2; no flush between steps",
+            "inputs": "weights N(0,0.02) drawn on the GPU from seeded generators, act_sq closed form"}
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha1()
+    for f in ("rq_gemv.cu", "rq_device.cuh"):
+        with open(os.path.join(ROOT, "weight_only_quantized_rq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[kernel]
+        return e["bytes_per_launch"] if e.get("source_hash") == kernel_hash() else None
+    except Exception:
+        return None
+
+
+# -------------------------------------------------------------- ours ------
+def run_ours(args, w, M):
+    import torch
+    import weight_only_quantized_rq_b200 as rq
+    from weight_only_quantized_rq_b200 import workloads as wl
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # CPU baseline first, before heavy GPU work (rank 0, single GPU only)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, desc, thr, _ = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": thr, "kind": "oracle", "sample": desc}
+
+    # pack the workload (not timed)
+    mats = []
+    for j, layer, m in w.matrices():
+        W = wl.weights(w, j, m, device=str(dev))
+        a = torch.from_numpy(wl.act_sq(w, m.K)).to(dev) if m.n_cand > 1 else None
+        p = rq.rq_quantize_pack(W, m.fmt, a, m.n_cand, 0.7 if m.n_cand > 1 else 1.0, 1.0)
+        mats.append((m, p))
+        del W
+    torch.cuda.synchronize()
+    # inputs: one device block holding every matrix's x, one for every y
+    xs_elems = sum(M * m.K for m, _ in mats)
+    ys_elems = sum(M * m.N for m, _ in mats)
+    xdev = torch.empty(xs_elems + 8 * len(mats), dtype=torch.bfloat16, device=dev)
+    ydev = torch.empty(ys_elems + 4 * len(mats), dtype=torch.float32, device=dev)
+    calls, xo, yo = [], 0, 0
+    for (m, p), (j, _, _) in zip(mats, w.matrices()):
+        x = xdev[xo:xo + M * m.K].view(M, m.K)
+        x.copy_(wl.activations(w, j, m.K, M, device=str(dev)))
+        y = ydev[yo:yo + M * m.N].view(M, m.N)
+        calls.append((x, p, y))
+        xo += (M * m.K + 7) // 8 * 8
+        yo += (M * m.N + 3) // 4 * 4
+    packed_bytes = sum(p.nbytes for _, p in mats)
+    alg_bytes = sum(p.nbytes + 2 * M * p.K + 4 * M * p.N for _, p in mats)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        for x, p, y in calls:
+            rq.rq_wgemm(x, p, y, stream=stream)
+
+    graph = None
+    with torch.cuda.stream(stream):
+        step()
+        stream.synchronize()
+        if not args.no_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+    torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            run()
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            run()
+        e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms], device=dev)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = ws * packed_bytes / (ms_max * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host x in, host y out
+    xh = torch.empty(xdev.shape, dtype=xdev.dtype, pin_memory=True)
+    yh = torch.empty(ydev.shape, dtype=ydev.dtype, pin_memory=True)
+    xh.copy_(xdev)
+    h2d = sum(M * m.K * 2 for m, _ in mats)
+    d2h = sum(M * m.N * 4 for m, _ in mats)
+
+    def e2e_step():
+        xdev.copy_(xh, non_blocking=True)
+        run()
+        yh.copy_(ydev, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms_e2e], device=dev)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_val = ws * packed_bytes / (float(t.item()) * 1e-3) / 1e9
+
+    status = rq.rq_device_status(stream)
+    hbm, src = peaks()
+    launches = len(calls)
+    per_launch_bytes = alg_bytes / launches
+    per_launch_s = ms * 1e-3 / launches
+    achieved = per_launch_bytes / per_launch_s / 1e9
+    traffic = recorded_traffic("gemv_w4g64_m1")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {**config_of(w, M), "packed_bytes_per_step": packed_bytes,
+                   "graph": graph is not None, "pdl": True,
+                   "parallelism": f"replicas{ws}" if ws > 1 else "single",
+                   "pct_hbm_measured": round(100 * value / ws / hbm, 2),
+                   "pct_hbm_nominal_8TBs": round(100 * value / ws / NOMINAL_HBM, 2)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic,
+                     "kernel": "gemv_kernel<w4g64, M=1>", "peak_source": src,
+                     "note": "average over the step's launches: algorithmic bytes (packed + x + y) / "
+                             "(step time / launches), launch gaps included"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        del graph
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    from weight_only_quantized_rq_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, args.M)
+    return run_ours(args, w, args.M)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

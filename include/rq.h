@@ -14,6 +14,9 @@
  *          tensor plus a scale tensor; summary paragraph: the kernels' output
  *          is bit-identical to the offline dequantization, and an int4 GEMV /
  *          small-M GEMM / tensor-core GEMM family serves batches up to 32.
+ *   [rwkv_quant_nv] "rwkv_quant_nv" project description, section "Operator
+ *          Optimization Details": decode tile shapes for the 4096x4096,
+ *          16384x4096 and 4096x16384 projections; r/k/v fused in one kernel.
  *
  * Conventions shared by every call:
  *   - W is stored [N][K] row-major (row n = output feature, K = input
@@ -152,6 +155,26 @@ int rq_quantize_pack(const float *W, int K, int N, const float *act_sq,
  * after writing the planes with your own kernel, synchronize or launch any
  * other kernel in between). Copies (cudaMemcpy*) are ordered as usual. */
 int rq_wgemm(const void *x, int M, int K, int N, const rq_packed *w, float *y, void *stream);
+
+/* One product of a batch: y = x * w_hat^T. */
+typedef struct rq_wgemm_item {
+    const void *x;          /* device bf16 [M][K] */
+    const rq_packed *w;     /* packed matrix (host descriptor) */
+    float *y;               /* device fp32 [M][N], overwritten */
+} rq_wgemm_item;
+
+/* `count` independent products in ONE launch, e.g. the r, k and v
+ * projections of a layer ([rwkv_quant_nv] "Operator Optimization Details":
+ * r/k/v computed in a single kernel). Every item has the same format and the
+ * same M; shapes may differ. The result equals `count` rq_wgemm calls. The
+ * launch's CTAs split the items' packed bytes evenly, so small matrices
+ * share the GPU instead of leaving it idle between launches.
+ *   items  host array of `count` items, 1 <= count <= 160
+ *   M      activation rows of every item, 1..128
+ * No y may overlap another item's y or any x. Same validation, status codes
+ * and ordering rules as rq_wgemm (the packed planes must not be written by
+ * the kernel launched just before this call on the stream). */
+int rq_wgemm_batch(const rq_wgemm_item *items, int count, int M, void *stream);
 
 /* Export w_hat as fp32 [N][K] into W_out (device).  ([CARD] summary: the
  * kernel output is bit-identical to the offline dequantization.) Uses the

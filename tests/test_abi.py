@@ -129,3 +129,26 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(rq, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(ImportError):
         rq.rq_version()
+
+
+def test_wgemm_batch_validation(L):
+    st = ctypes.c_void_p(0)
+    d1 = _desc("w4g64", 2048, 256)
+    d2 = _desc("w8g16", 2048, 256)
+    Items = rq.RqWgemmItem * 2
+    good = Items(rq.RqWgemmItem(0x40000, ctypes.pointer(d1), 0x50000),
+                 rq.RqWgemmItem(0x60000, ctypes.pointer(d1), 0x70000))
+    assert L.rq_wgemm_batch(None, 1, 1, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_wgemm_batch(good, 0, 1, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_wgemm_batch(good, 161, 1, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_wgemm_batch(good, 2, 0, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_wgemm_batch(good, 2, 129, st) == rq.RQ_ERR_INVALID_ARG
+    mixed = Items(rq.RqWgemmItem(0x40000, ctypes.pointer(d1), 0x50000),
+                  rq.RqWgemmItem(0x60000, ctypes.pointer(d2), 0x70000))
+    assert L.rq_wgemm_batch(mixed, 2, 1, st) == rq.RQ_ERR_FORMAT_MISMATCH
+    mis = Items(rq.RqWgemmItem(0x40000, ctypes.pointer(d1), 0x50000),
+                rq.RqWgemmItem(0x60008, ctypes.pointer(d1), 0x70000))
+    assert L.rq_wgemm_batch(mis, 2, 1, st) == rq.RQ_ERR_MISALIGNED
+    nul = Items(rq.RqWgemmItem(0x40000, ctypes.pointer(d1), 0x50000),
+                rq.RqWgemmItem(0x60000, None, 0x70000))
+    assert L.rq_wgemm_batch(nul, 2, 1, st) == rq.RQ_ERR_INVALID_ARG

@@ -291,3 +291,50 @@ def _full_size_check(widx, layer_sample=1, rows_per_matrix=48, Ms=None):
 @pytest.mark.parametrize("widx", [0, 1, 2, 3, 4])
 def test_full_size_workloads_sampled(widx):
     _full_size_check(widx)
+
+
+# --------------------------------------------------------------- batches ---
+@pytest.mark.parametrize("fmt,shapes,M", [
+    ("w4g64", [(2048, 2048), (2048, 8192), (8192, 2048), (768, 5), (2048, 1)], 1),
+    ("w4g64", [(1024, 300), (1024, 64), (4096, 77)], 2),
+    ("w8g16", [(2048, 130), (4096, 33), (448, 9)], 1),
+    ("w4sb32", [(2560, 200), (10240, 40), (256, 3)], 3),
+])
+def test_wgemm_batch_matches_oracle(fmt, shapes, M):
+    """One launch over products of different shapes equals the oracle per
+    product; outputs are written only inside each y (guard bands)."""
+    xs, ws, ys, refs = [], [], [], []
+    bigs = []
+    for i, (K, N) in enumerate(shapes):
+        W = wl.random_matrix(700 + i, N, K).numpy()
+        oc, osc = oracle.pack(fmt, W, None, n_cand=4)
+        p = upload(fmt, K, N, oc, osc)
+        x, xb = make_x(800 + i, M, K)
+        big = torch.full((M * N + 512,), float("nan"), device="cuda")
+        xs.append(x.cuda())
+        ws.append(p)
+        ys.append(big[256:256 + M * N].view(M, N))
+        bigs.append((big, M * N))
+        refs.append((oracle.wgemm(fmt, xb, K, N, oc, osc), xb, oracle.dequant(fmt, K, N, oc, osc)))
+    rq.rq_wgemm_batch(xs, ws, ys)
+    torch.cuda.synchronize()
+    for y, (y_ref, xb, wd), (big, n) in zip(ys, refs, bigs):
+        check_y(y.cpu().numpy(), y_ref, xb, wd)
+        assert bool(torch.isnan(big[:256]).all()) and bool(torch.isnan(big[256 + n:]).all())
+
+
+def test_wgemm_batch_equals_single_calls():
+    """The batched launch gives bit-identical outputs to one call per item
+    (each row's sum is formed by the same lanes in the same order)."""
+    fmt, M = "w4g64", 1
+    shapes = [(2048, 2048)] * 3 + [(2048, 8192), (8192, 2048)]
+    xs, ws = [], []
+    for i, (K, N) in enumerate(shapes):
+        ws.append(rq.rq_quantize_pack(wl.random_matrix(900 + i, N, K).cuda(), fmt))
+        xs.append(make_x(950 + i, M, K)[0].cuda())
+    ys = [torch.empty(M, w.N, device="cuda") for w in ws]
+    rq.rq_wgemm_batch(xs, ws, ys)
+    singles = [rq.rq_wgemm(x, w) for x, w in zip(xs, ws)]
+    torch.cuda.synchronize()
+    for a, b in zip(ys, singles):
+        assert torch.equal(a, b)

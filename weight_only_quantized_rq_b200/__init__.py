@@ -34,8 +34,9 @@ RQ_W4_SYM_G64 = 1
 RQ_W8_SYM_G16 = 2
 RQ_W4_ASYM_SB32 = 3
 FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_ASYM_SB32}
-EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_dequant", "rq_status_string",
-           "rq_last_cuda_error", "rq_device_status", "rq_version")
+EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_dequant",
+           "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
+MAX_BATCH = 160
 
 
 class RqSearch(ctypes.Structure):
@@ -45,6 +46,10 @@ class RqSearch(ctypes.Structure):
 class RqPacked(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int), ("K", ctypes.c_int), ("N", ctypes.c_int), ("reserved", ctypes.c_int),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class RqWgemmItem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("w", ctypes.POINTER(RqPacked)), ("y", ctypes.c_void_p)]
 
 
 class RqError(RuntimeError):
@@ -75,6 +80,8 @@ def _lib() -> ctypes.CDLL:
         L.rq_quantize_pack.restype = I
         L.rq_wgemm.argtypes = [P, I, I, I, ctypes.POINTER(RqPacked), P, P]
         L.rq_wgemm.restype = I
+        L.rq_wgemm_batch.argtypes = [ctypes.POINTER(RqWgemmItem), I, I, P]
+        L.rq_wgemm_batch.restype = I
         L.rq_dequant.argtypes = [ctypes.POINTER(RqPacked), P, P]
         L.rq_dequant.restype = I
         L.rq_status_string.argtypes = [I]
@@ -181,6 +188,32 @@ def rq_wgemm(x: torch.Tensor, w: Packed, y: torch.Tensor | None = None, stream=N
     return y
 
 
+class WgemmBatch:
+    """A prepared batch for rq_wgemm_batch: the ctypes item array is built
+    once (so repeated calls and CUDA-graph capture pay no marshalling)."""
+
+    def __init__(self, xs, ws, ys):
+        if not (len(xs) == len(ws) == len(ys)) or not 1 <= len(xs) <= MAX_BATCH:
+            raise ValueError("need 1..160 items with one x, w, y each")
+        self.M = int(xs[0].shape[0])
+        self._keep = (list(xs), list(ws), list(ys))
+        self._descs = [w.desc() for w in ws]
+        self._items = (RqWgemmItem * len(xs))()
+        for i, (x, d, y) in enumerate(zip(xs, self._descs, ys)):
+            if int(x.shape[0]) != self.M:
+                raise ValueError("every item must have the same M")
+            self._items[i] = RqWgemmItem(x.data_ptr(), ctypes.pointer(d), y.data_ptr())
+        self.count = len(xs)
+
+    def __call__(self, stream=None):
+        _check(_lib().rq_wgemm_batch(self._items, self.count, self.M, _stream(stream)), "rq_wgemm_batch")
+
+
+def rq_wgemm_batch(xs, ws, ys, stream=None) -> None:
+    """Independent products ys[i] = xs[i] @ w_hat_i.T in one launch."""
+    WgemmBatch(xs, ws, ys)(stream)
+
+
 def rq_dequant(w: Packed, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """w_hat as fp32 [N][K] (CUDA)."""
     if out is None:
@@ -202,5 +235,6 @@ def rq_device_status(stream=None) -> int:
 # short aliases
 quantize_pack = rq_quantize_pack
 wgemm = rq_wgemm
+wgemm_batch = rq_wgemm_batch
 dequant = rq_dequant
 packed_size = rq_packed_size

@@ -100,7 +100,23 @@ int rq_wgemm(const void* x, int M, int K, int N, const rq_packed* w, float* y, v
     if (s != RQ_OK) return s;
     if (!aligned16(x) || !aligned16(y)) return RQ_ERR_MISALIGNED;
     rq::WgemmArgs a = {w->fmt, M, K, N, x, w->codes, w->scales, y};
-    return cuda_status(rq::launch_gemv(a, static_cast<cudaStream_t>(stream)));
+    return cuda_status(rq::launch_gemv(&a, 1, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
+    if (!items || count < 1 || count > rq::kMaxBatch) return RQ_ERR_INVALID_ARG;
+    if (M < 1 || M > 128) return RQ_ERR_INVALID_ARG;
+    rq::WgemmArgs a[rq::kMaxBatch];
+    for (int i = 0; i < count; ++i) {
+        const rq_wgemm_item& it = items[i];
+        if (!it.x || !it.y || !it.w) return RQ_ERR_INVALID_ARG;
+        int s = check_packed(it.w, it.w->K, it.w->N);
+        if (s != RQ_OK) return s;
+        if (it.w->fmt != items[0].w->fmt) return RQ_ERR_FORMAT_MISMATCH;
+        if (!aligned16(it.x) || !aligned16(it.y)) return RQ_ERR_MISALIGNED;
+        a[i] = {it.w->fmt, M, it.w->K, it.w->N, it.x, it.w->codes, it.w->scales, it.y};
+    }
+    return cuda_status(rq::launch_gemv(a, count, static_cast<cudaStream_t>(stream)));
 }
 
 int rq_dequant(const rq_packed* w, float* W_out, void* stream) {

@@ -126,6 +126,34 @@ __device__ __forceinline__ float4 lds128f(const void* p) {
     return v;
 }
 
+// Loads from 32-bit shared-memory addresses (no generic-to-shared conversion
+// per access). Volatile keeps them after the barrier waits that guard them.
+__device__ __forceinline__ uint4 lds128_a(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float4 lds128f_a(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32_a(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16_a(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float ldsf_a(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+
 // --------------------------------------------------------------- unpack ---
 // int4 codes. A 32-bit word holds eight nibbles; nibble p (bits 4p..4p+3)
 // is the code of weight k = 8i + p of that word (byte j: k = 2j low, 2j+1
@@ -158,6 +186,95 @@ __device__ __forceinline__ void unpack_w4(uint32_t w, float f[8]) {
 }
 // Position inside the word of output slot j of unpack_w4.
 __host__ __device__ constexpr int w4_slot_nibble(int j) { return j < 4 ? 2 * j : 2 * (j - 4) + 1; }
+
+// int4 codes as bf16 pairs (the GEMV and dequant unpack). Pair j (0..3) of a
+// word holds nibble j in its low half and nibble j+4 in its high half, each
+// as the bf16 value 128 + u: the nibble lands in mantissa bits 0..3 under the
+// exponent pattern 0x43 (bf16 128.0, mantissa bit 0 weighs 1). One shift and
+// one three-input logic op per two weights.
+constexpr uint32_t kW4PairMagic = 0x43004300u;
+
+template <int J>
+__device__ __forceinline__ uint32_t w4_pair(uint32_t w) {
+    uint32_t d;
+    const uint32_t v = J ? (w >> (4 * J)) : w;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(v), "r"(0x000F000Fu), "r"(kW4PairMagic));  // (v & m) | c
+    return d;
+}
+
+// fp32 value of the low / high bf16 half of a 32-bit word (exact).
+__device__ __forceinline__ float bf16lo_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// c + a.half(AH) * b.half(BH), with bf16 operands and an fp32 accumulator:
+// the product of two bf16 values is exact in fp32, so this equals an fp32
+// fma of the two values widened to fp32 (one rounding).
+template <int AH, int BH>
+__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
+    float d;
+    if (AH == 0 && BH == 0)
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.bf16 %0, a0, b0, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if (AH == 1 && BH == 0)
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.bf16 %0, a1, b0, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if (AH == 0 && BH == 1)
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.bf16 %0, a0, b1, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.bf16 %0, a1, b1, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+// The eight values 128 + u_k of one code word, in natural k order, widened
+// exactly from the bf16 pairs the GEMV multiplies (rq_dequant's unpack).
+__device__ __forceinline__ void w4_word_values(uint32_t w, float o[8]) {
+    const uint32_t r0 = w4_pair<0>(w), r1 = w4_pair<1>(w), r2 = w4_pair<2>(w), r3 = w4_pair<3>(w);
+    o[0] = bf16lo_f32(r0); o[4] = bf16hi_f32(r0);
+    o[1] = bf16lo_f32(r1); o[5] = bf16hi_f32(r1);
+    o[2] = bf16lo_f32(r2); o[6] = bf16hi_f32(r2);
+    o[3] = bf16lo_f32(r3); o[7] = bf16hi_f32(r3);
+}
+
+// acc[0..NA-1] += the 8 products (128 + u_k) * x_k of one code word, spread
+// over NA independent accumulators (NA = 8: one per position, no chain
+// inside a word; NA = 4 or 2: products folded pairwise).
+template <int NA>
+__device__ __forceinline__ void dot8_w4_split(uint32_t w, uint4 X, float (&acc)[NA]) {
+    const uint32_t r0 = w4_pair<0>(w), r1 = w4_pair<1>(w), r2 = w4_pair<2>(w), r3 = w4_pair<3>(w);
+    acc[0 % NA] = fma_bf16<0, 0>(r0, X.x, acc[0 % NA]);   // u0 x0
+    acc[1 % NA] = fma_bf16<1, 0>(r0, X.z, acc[1 % NA]);   // u4 x4
+    acc[2 % NA] = fma_bf16<0, 1>(r1, X.x, acc[2 % NA]);   // u1 x1
+    acc[3 % NA] = fma_bf16<1, 1>(r1, X.z, acc[3 % NA]);   // u5 x5
+    acc[4 % NA] = fma_bf16<0, 0>(r2, X.y, acc[4 % NA]);   // u2 x2
+    acc[5 % NA] = fma_bf16<1, 0>(r2, X.w, acc[5 % NA]);   // u6 x6
+    acc[6 % NA] = fma_bf16<0, 1>(r3, X.y, acc[6 % NA]);   // u3 x3
+    acc[7 % NA] = fma_bf16<1, 1>(r3, X.w, acc[7 % NA]);   // u7 x7
+}
+
+template <int NA>
+__device__ __forceinline__ float sum_acc(const float (&a)[NA]) {
+    if (NA == 8) return ((a[0 % NA] + a[1 % NA]) + (a[2 % NA] + a[3 % NA])) + ((a[4 % NA] + a[5 % NA]) + (a[6 % NA] + a[7 % NA]));
+    if (NA == 4) return (a[0 % NA] + a[1 % NA]) + (a[2 % NA] + a[3 % NA]);
+    if (NA == 2) return a[0] + a[1 % NA];
+    return a[0];
+}
+
+// acc += sum over the 8 weights of one code word of (128 + u_k) * x_k, where
+// X0..X3 hold x_0..x_7 as natural-order bf16 pairs ((x0,x1), (x2,x3), ...).
+__device__ __forceinline__ float dot8_w4(uint32_t w, uint4 X, float acc) {
+    const uint32_t r0 = w4_pair<0>(w), r1 = w4_pair<1>(w), r2 = w4_pair<2>(w), r3 = w4_pair<3>(w);
+    acc = fma_bf16<0, 0>(r0, X.x, acc);   // u0 x0
+    acc = fma_bf16<1, 0>(r0, X.z, acc);   // u4 x4
+    acc = fma_bf16<0, 1>(r1, X.x, acc);   // u1 x1
+    acc = fma_bf16<1, 1>(r1, X.z, acc);   // u5 x5
+    acc = fma_bf16<0, 0>(r2, X.y, acc);   // u2 x2
+    acc = fma_bf16<1, 0>(r2, X.w, acc);   // u6 x6
+    acc = fma_bf16<0, 1>(r3, X.y, acc);   // u3 x3
+    acc = fma_bf16<1, 1>(r3, X.w, acc);   // u7 x7
+    return acc;
+}
 
 // int8 codes. Byte k of a word is the code u = q + 128 of weight k. Each byte
 // is placed in bits 8..15 under exponent byte 0x47 (fp32 32768.0, mantissa

@@ -1,70 +1,306 @@
 // rq_gemv.cu -- the memory-bound product y = x * w_hat^T for a few activation
-// rows (decode), with w_hat formed in registers.
+// rows (decode), with w_hat formed in registers; one launch may carry a batch
+// of independent products (e.g. the r, k, v projections of a layer).
 //
-// Source: RWKV-7 G1 1.5B int4 model card, summary paragraph: decode is served
-// by a hand-written int4 GEMV / small-M GEMM family and the kernel output is
-// bit-identical to the offline dequantization; rwkv-quant article, "Two
-// presets and six sizes": the int8 group-16 and int4 superblock formats.
+// Sources: RWKV-7 G1 1.5B int4 model card, summary paragraph: decode is
+// served by a hand-written int4 GEMV / small-M GEMM family and the kernel
+// output is bit-identical to the offline dequantization. rwkv-quant article,
+// "Two presets and six sizes": the int8 group-16 and int4 superblock formats.
+// rwkv_quant_nv project description, "Operator Optimization Details": the
+// r/k/v projections computed in a single kernel.
 //
 // Design (B200):
-//  * One producer warp streams whole row tiles (R rows x K, codes and scales
-//    are contiguous in HBM) into a ring of shared-memory stages with
-//    untiled bulk-async copies completed on mbarriers; the copies are issued
-//    before griddepcontrol.wait, so with programmatic dependent launch the
-//    next matrix's weights are already in flight while the previous kernel
-//    drains.
-//  * x is staged once per CTA as fp32 in shared memory, in the order the
-//    unpack produces weights, interleaved by 16-byte quads so that lanes
-//    reading consecutive half-chunks hit consecutive banks; the sum of x over
-//    each 32-weight half-chunk is stored beside it.
-//  * A team of T lanes (a power of two dividing K/32) owns RW rows of a tile;
-//    lane i of the team takes half-chunks i, i+T, ... of those rows. Codes are
-//    unpacked to fp32 values 128 + u (or q for int8) with byte permutes and
-//    multiplied into fp32 accumulators; the per-group scale and the code
-//    offset are applied once per half-chunk:
-//        sum_k (u_k - 8) x_k s = s * (sum_k (128 + u_k) x_k - 136 sum_k x_k).
-//  * Team partial sums are reduced with warp shuffles and written once.
+//  * The products of a launch are laid end to end on one axis of packed
+//    bytes; CTA c (one per SM) owns a contiguous, balanced stretch of it, i.e.
+//    contiguous row ranges of one or a few products. Codes and scales of
+//    consecutive rows are contiguous in HBM, so a group of rows is one
+//    untiled bulk-async copy per plane into a shared-memory stage, completed
+//    on an mbarrier. A producer warp keeps the ring full, starting before
+//    griddepcontrol.wait: with programmatic dependent launch the weights
+//    stream in while the previous kernel finishes.
+//  * After the wait, each product's x is staged in shared memory, interleaved
+//    by 16-byte quads so that lanes reading consecutive half-chunks (32
+//    weights) hit consecutive banks, with the sum of x over each half-chunk.
+//  * A team of T lanes (a power of two dividing K/32) owns RW rows of a group;
+//    lane i takes half-chunks i, i+T, ... of those rows.
+//    int4: one shift + one lop3 turns two nibbles into the bf16 pair
+//    (128 + u, 128 + u'), multiplied by bf16 x with fp32-accumulating
+//    fma.rn.f32.bf16; the scale and code offset are applied once per
+//    half-chunk:  sum_k (u_k - 8) x_k s = s (sum_k (128 + u_k) x_k - 136 sum_k x_k).
+//    int8: a byte permute places each code under an fp32 exponent (32768 + u),
+//    one subtraction gives q exactly, fp32 fma with fp32 x.
+//  * Team partial sums are reduced with warp shuffles; one store per output.
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "rq_device.cuh"
 #include "rq_internal.h"
 
+// Phase marks for external profiling builds; no code in this library.
+#ifndef RQ_PHASE_MARK
+#define RQ_PHASE_MARK(i)
+#endif
+
 namespace rq {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
+#ifndef RQ_GEMV_WARPS
+#define RQ_GEMV_WARPS 8
+#endif
+constexpr int kConsumerWarps = RQ_GEMV_WARPS;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
 
-struct GemvParams {
-    const uint16_t* x;     // bf16 bits [M][K]
+struct Item {                  // one product of a launch
+    const uint16_t* x;         // bf16 bits [M][K]
     const uint8_t* codes;
     const uint8_t* scales;
-    float* y;
+    float* y;                  // fp32 [M][N]
+    long long cost0;           // packed bytes of the items before this one
     int K, N;
-    int m0, mrows;         // activation rows [m0, m0 + mrows) handled here
-    int T, HJ, RW, R;      // team lanes, half-chunks per lane, rows per team, rows per tile
-    int stages, tiles;
-    uint32_t crb, srb;     // code / scale bytes per row
-    uint32_t stage_bytes, scale_off;
-    uint32_t x_off, bar_off;
+    int T, HJ;                 // team lanes, half-chunks per lane
+    int RW, Rg;                // rows per team, rows per group (a multiple of rho)
+    int rho;                   // rows per unit; a unit is the grain of the CTA split
+    uint32_t crb, srb;         // code / scale bytes per row
+    uint32_t ucost;            // bytes of one unit (rho rows of both planes)
 };
 
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+template <int MAXI>
+struct Batch {
+    int count, m0, mrows;      // items; activation rows [m0, m0 + mrows) of every item
+    int stages;
+    long long total;           // packed bytes of all items
+    uint32_t stage_bytes, x_off, xsum_off, bar_off;
+    Item it[MAXI];
+};
 
+// Units [ua, ub) of item `it` that start inside the cost range [lo, hi).
+__device__ __forceinline__ void item_units(const Item& it, long long lo, long long hi, int& ua, int& ub) {
+    const long long U = (it.N + it.rho - 1) / it.rho;
+    auto first_at_or_after = [&](long long c) -> long long {
+        const long long d = c - it.cost0;
+        if (d <= 0) return 0;
+        const long long u = (d + it.ucost - 1) / it.ucost;
+        return u < U ? u : U;
+    };
+    ua = (int)first_at_or_after(lo);
+    ub = (int)first_at_or_after(hi);
+}
+
+template <int FMT, int MT>
+__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xbuf, float* xsum, int tid) {
+    constexpr bool kW4 = FMT != kFmtW8G16;
+    const int hcpr = it.K >> 5;
+    for (int i = tid; i < MT * hcpr; i += kConsumerWarps * 32) {
+        const int m = i / hcpr, h = i - m * hcpr;
+        uint4 v[4] = {};
+        if (m < mrows) {
+            const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)h * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
+        }
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
+        if (kW4) {   // bf16 quads, natural order: quad q = x[8q .. 8q+7]
+            uint4* dst = reinterpret_cast<uint4*>(xbuf) + (size_t)m * 4 * hcpr + h;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[q];
+        } else {     // fp32 quads, natural order: quad q = x[4q .. 4q+3]
+            float4* dst = reinterpret_cast<float4*>(xbuf) + (size_t)m * 8 * hcpr + h;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                dst[(size_t)q * hcpr] = make_float4(bf16lo_f32(w[2 * q]), bf16hi_f32(w[2 * q]),
+                                                    bf16lo_f32(w[2 * q + 1]), bf16hi_f32(w[2 * q + 1]));
+        }
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+            s0 += bf16lo_f32(w[j]) + bf16hi_f32(w[j]);
+            s1 += bf16lo_f32(w[j + 1]) + bf16hi_f32(w[j + 1]);
+        }
+        xsum[(size_t)m * hcpr + h] = s0 + s1;
+    }
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& c, int i) {
+    return i == 0 ? c.x : i == 1 ? c.y : i == 2 ? c.z : c.w;
+}
+
+// One group of rows of item `it` in the stage at shared address st_s: this
+// team's rows rbase .. rbase + RW - 1 of the group; writes their outputs.
+// Rows past rg (the group's last rows) lie inside the stage buffer, which
+// always has room for Rg rows; they hold stale bytes whose results are never
+// stored.
 template <int FMT, int MT, int RW>
-__global__ void __launch_bounds__(kGemvThreads)
-gemv_kernel(const GemvParams p) {
+__device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s,
+                                           uint32_t xsum_s, int m0, int mrows, int lane, int rbase) {
+    constexpr bool kW4 = FMT != kFmtW8G16;
+    constexpr int U = RW == 1 ? 2 : 1;                   // half-chunks per iteration
+    const int hcpr = it.K >> 5, T = it.T, HJ = it.HJ;
+    const int li = lane & (T - 1);
+    const uint32_t crb = it.crb, srb = it.srb;
+    const uint32_t ssc_s = st_s + (uint32_t)round16((size_t)it.Rg * crb);
+    // x quads: (m * Q + q) * hcpr + h, Q = 4 (bf16) or 8 (fp32) quads per half-chunk
+    const uint32_t xstride = (uint32_t)hcpr * 16u;
+    const uint32_t xa0 = x_s + (uint32_t)li * 16u;
+    const uint32_t xs0 = xsum_s + (uint32_t)li * 4u;
+    float yacc[RW][MT];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) yacc[r][m] = 0.0f;
+
+    if (kW4) {
+        // W4G64: codes at row * crb + h * 16, scale at (h / 2) * 2.
+        // W4SB32: record at row * crb + (h / 8) * 144; T is a multiple of 8
+        // (K % 256 == 0), so a lane always sees the same group j = li % 8.
+        const int j = li & 7;
+        uint32_t ca[RW], sa[RW];
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            if (FMT == kFmtW4G64) {
+                ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)li * 16u;
+                sa[r] = ssc_s + (uint32_t)(rbase + r) * srb + (uint32_t)(li >> 1) * 2u;
+            } else {
+                ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)(li >> 3) * 144u;
+                sa[r] = 0u;
+            }
+        }
+        // four accumulators per row and m, whatever the launch shape, so a row's
+        // sums (and results) do not depend on RW or on batching
+        constexpr int NA = 4;
+        for (int hj = 0; hj < HJ; hj += U) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (u > 0 && hj + u >= HJ) break;
+                const uint32_t dh = (uint32_t)(hj + u) * (uint32_t)T;
+                float xsm[MT];
+#pragma unroll
+                for (int m = 0; m < MT; ++m) xsm[m] = ldsf_a(xs0 + (uint32_t)m * (uint32_t)hcpr * 4u + dh * 4u);
+                uint4 c[RW];
+                float sA[RW], sB[RW];
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    if (FMT == kFmtW4G64) {
+                        c[r] = lds128_a(ca[r] + dh * 16u);
+                        sA[r] = __half2float(__ushort_as_half((unsigned short)lds16_a(sa[r] + dh)));
+                        sB[r] = 0.0f;
+                    } else {
+                        const uint32_t rec = ca[r] + (dh >> 3) * 144u;
+                        const uint4 hd = lds128_a(rec);
+                        c[r] = lds128_a(rec + 16u + (uint32_t)j * 16u);
+                        const float d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xffffu)));
+                        const float dm = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
+                        sA[r] = __fmul_rn(d, (float)sb_field(hd.y, hd.z, hd.w, 0, j));
+                        sB[r] = __fmul_rn(dm, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
+                    }
+                }
+                float acc[RW][MT][NA];
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+#pragma unroll
+                        for (int k = 0; k < NA; ++k) acc[r][m][k] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        const uint4 X = lds128_a(xa0 + dh * 16u + (uint32_t)(m * 4 + i) * xstride);
+#pragma unroll
+                        for (int r = 0; r < RW; ++r) dot8_w4_split<NA>(word_of(c[r], i), X, acc[r][m]);
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        const float a = sum_acc<NA>(acc[r][m]);
+                        if (FMT == kFmtW4G64) {
+                            yacc[r][m] = fmaf(sA[r], fmaf(-136.0f, xsm[m], a), yacc[r][m]);
+                        } else {
+                            yacc[r][m] = fmaf(sA[r], fmaf(-128.0f, xsm[m], a), yacc[r][m]);
+                            yacc[r][m] = fmaf(-sB[r], xsm[m], yacc[r][m]);
+                        }
+                    }
+            }
+        }
+    } else {
+        // int8 group 16: 32 code bytes per row and half-chunk = groups 2h, 2h+1;
+        // x as fp32 quads, 8 per half-chunk
+        uint32_t ca[RW], sa[RW];
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)li * 32u;
+            sa[r] = ssc_s + (uint32_t)(rbase + r) * srb + (uint32_t)li * 4u;
+        }
+        for (int hj = 0; hj < HJ; hj += U) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (u > 0 && hj + u >= HJ) break;
+                const uint32_t dh = (uint32_t)(hj + u) * (uint32_t)T;
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    const uint4 c0 = lds128_a(ca[r] + dh * 32u);
+                    const uint4 c1 = lds128_a(ca[r] + dh * 32u + 16u);
+                    const uint32_t sp = lds32_a(sa[r] + dh * 4u);
+                    const float s0 = __half2float(__ushort_as_half((unsigned short)(sp & 0xffffu)));
+                    const float s1 = __half2float(__ushort_as_half((unsigned short)(sp >> 16)));
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        float a[MT];
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) a[m] = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            float f[4];
+                            unpack_w8(word_of(g ? c1 : c0, i), f);
+#pragma unroll
+                            for (int m = 0; m < MT; ++m) {
+                                const float4 xv = lds128f_a(xa0 + dh * 16u + (uint32_t)(m * 8 + g * 4 + i) * xstride);
+                                a[m] = fmaf(f[0], xv.x, a[m]);
+                                a[m] = fmaf(f[1], xv.y, a[m]);
+                                a[m] = fmaf(f[2], xv.z, a[m]);
+                                a[m] = fmaf(f[3], xv.w, a[m]);
+                            }
+                        }
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) yacc[r][m] = fmaf(g ? s1 : s0, a[m], yacc[r][m]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float v = yacc[r][m];
+            for (int o = T >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            yacc[r][m] = v;
+        }
+    if (li == 0) {
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int rr = rbase + r;
+            if (rr < rg)
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+                    if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = yacc[r][m];
+        }
+    }
+}
+
+template <int FMT, int MT, int MAXI>
+__global__ void __launch_bounds__(kThreads, kConsumerWarps > 8 ? 1 : (MT == 1 ? 3 : 2))
+gemv_kernel(const Batch<MAXI> p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int hcpr = p.K >> 5;                       // half-chunks (32 weights) per row
-    float* xs = reinterpret_cast<float*>(smem + p.x_off);   // [MT][8][hcpr] float4
-    float* xsum = xs + (size_t)MT * p.K;                    // [MT][hcpr]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
     uint64_t* empty = full + p.stages;
+    uint8_t* xbuf = smem + p.x_off;
+    float* xsum = reinterpret_cast<float*>(smem + p.xsum_off);
+    const long long lo = (long long)blockIdx.x * p.total / gridDim.x;
+    const long long hi = (long long)(blockIdx.x + 1) * p.total / gridDim.x;
 
-    const int my_tiles = (int)blockIdx.x < p.tiles ? (p.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     if (tid == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1);
@@ -74,241 +310,96 @@ gemv_kernel(const GemvParams p) {
     }
     __syncthreads();
     grid_dep_launch();
+    RQ_PHASE_MARK(0);
 
-    if (warp == kConsumerWarps) {                    // producer warp
+    if (warp == kConsumerWarps) {                        // producer warp
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();
-            for (int i = 0; i < my_tiles; ++i) {
-                const int s = i % p.stages;
-                if (i >= p.stages && !mbar_wait_bounded(&empty[s], ((i / p.stages) - 1) & 1, kStatusSlotWait))
-                    break;
-                const int n0 = ((int)blockIdx.x + i * (int)gridDim.x) * p.R;
-                const int rows = min(p.R, p.N - n0);
-                const uint32_t cb = (uint32_t)rows * p.crb;
-                const uint32_t sb = p.srb ? (((uint32_t)rows * p.srb + 15u) & ~15u) : 0u;
-                uint8_t* st = smem + (size_t)s * p.stage_bytes;
-                mbar_arrive_expect_tx(&full[s], cb + sb);
-                bulk_g2s(st, p.codes + (size_t)n0 * p.crb, cb, &full[s], pol);
-                if (sb) bulk_g2s(st + p.scale_off, p.scales + (size_t)n0 * p.srb, sb, &full[s], pol);
+            int gi = 0;
+            bool ok = true;
+            for (int i = 0; i < p.count && ok; ++i) {
+                const Item& it = p.it[i];
+                int ua, ub;
+                item_units(it, lo, hi, ua, ub);
+                const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
+                for (int g0 = ra; g0 < rb; g0 += it.Rg, ++gi) {
+                    const int s = gi % p.stages;
+                    if (gi >= p.stages && !mbar_wait_bounded(&empty[s], ((gi / p.stages) - 1) & 1, kStatusSlotWait)) {
+                        ok = false;
+                        break;
+                    }
+                    const int rg = min(it.Rg, rb - g0);
+                    const uint32_t cb = (uint32_t)rg * it.crb;
+                    const uint32_t sb = it.srb ? (((uint32_t)rg * it.srb + 15u) & ~15u) : 0u;
+                    uint8_t* st = smem + (size_t)s * p.stage_bytes;
+                    mbar_arrive_expect_tx(&full[s], cb + sb);
+                    bulk_g2s(st, it.codes + (size_t)g0 * it.crb, cb, &full[s], pol);
+                    if (sb)
+                        bulk_g2s(st + round16((size_t)it.Rg * it.crb), it.scales + (size_t)g0 * it.srb, sb, &full[s], pol);
+                }
             }
         }
         return;
     }
 
-    // ---- consumers: stage x (it is written by the previous kernel) --------
-    grid_dep_wait();
-    for (int i = tid; i < MT * hcpr; i += kConsumerWarps * 32) {
-        const int m = i / hcpr, h = i - m * hcpr;
-        uint4 v[4] = {};
-        if (m < p.mrows) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)(p.m0 + m) * p.K + (size_t)h * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
-        }
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(v);  // 16 words = 32 bf16, natural order
-        float4* dst = reinterpret_cast<float4*>(xs) + (size_t)m * 8 * hcpr + h;
-        float sum = 0.0f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            float4 f;
-            if (FMT == kFmtW8G16) {          // natural order: weights 4q..4q+3
-                f = make_float4(bf_lo(w[2 * q]), bf_hi(w[2 * q]), bf_lo(w[2 * q + 1]), bf_hi(w[2 * q + 1]));
-            } else {                          // int4 slot order: word q/2, even (q even) or odd weights
-                const uint32_t* ww = w + 4 * (q >> 1);
-                f = (q & 1) ? make_float4(bf_hi(ww[0]), bf_hi(ww[1]), bf_hi(ww[2]), bf_hi(ww[3]))
-                            : make_float4(bf_lo(ww[0]), bf_lo(ww[1]), bf_lo(ww[2]), bf_lo(ww[3]));
+    // ---- consumers ---------------------------------------------------------
+    const uint32_t smem_s = smem_u32(smem);
+    grid_dep_wait();                                     // x is written by the previous kernel
+    RQ_PHASE_MARK(1);
+    int gi = 0;
+    bool first = true;
+    for (int i = 0; i < p.count; ++i) {
+        const Item& it = p.it[i];
+        int ua, ub;
+        item_units(it, lo, hi, ua, ub);
+        const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
+        if (ra >= rb) continue;
+        if (!first) asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
+        first = false;
+        stage_x<FMT, MT>(it, p.m0, p.mrows, xbuf, xsum, tid);
+        asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
+        RQ_PHASE_MARK(2);
+        const int T = it.T, RW = it.RW;
+        const int team = lane / T;
+        const int rbase = (warp * (32 / T) + team) * RW;      // first row of this team in a group
+        const int wfirst = warp * (32 / T) * RW;               // first row of this warp in a group
+        for (int g0 = ra; g0 < rb; g0 += it.Rg, ++gi) {
+            const int s = gi % p.stages;
+            if (!mbar_wait_bounded(&full[s], (gi / p.stages) & 1, kStatusTmaWait)) return;
+            RQ_PHASE_MARK(3);
+            const int rg = min(it.Rg, rb - g0);
+            if (wfirst < rg) {                           // warp-uniform
+                const uint32_t st_s = smem_s + (uint32_t)s * p.stage_bytes;
+                if (RW == 4)
+                    gemv_group<FMT, MT, 4>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows, lane, rbase);
+                else if (RW == 2)
+                    gemv_group<FMT, MT, 2>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows, lane, rbase);
+                else
+                    gemv_group<FMT, MT, 1>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows, lane, rbase);
             }
-            dst[(size_t)q * hcpr] = f;
-            sum += (f.x + f.y) + (f.z + f.w);
-        }
-        xsum[(size_t)m * hcpr + h] = sum;
-    }
-    asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
-
-    const int T = p.T;
-    const int team = lane / T, li = lane - team * T;
-    const int rbase = (warp * (32 / T) + team) * RW;
-    bool ok = true;
-
-    for (int it = 0; it < my_tiles; ++it) {
-        const int s = it % p.stages;
-        if (!mbar_wait_bounded(&full[s], (it / p.stages) & 1, kStatusTmaWait)) { ok = false; break; }
-        const int n0 = ((int)blockIdx.x + it * (int)gridDim.x) * p.R;
-        const int rows = min(p.R, p.N - n0);
-        const uint8_t* st = smem + (size_t)s * p.stage_bytes;
-        const uint8_t* ssc = st + p.scale_off;
-
-        float yacc[RW][MT];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < MT; ++m) yacc[r][m] = 0.0f;
-
-        for (int hj = 0; hj < p.HJ; ++hj) {
-            const int h = li + T * hj;
-            float xsm[MT];
-#pragma unroll
-            for (int m = 0; m < MT; ++m) xsm[m] = xsum[(size_t)m * hcpr + h];
-            const float4* xq = reinterpret_cast<const float4*>(xs) + h;
-
-            if (FMT == kFmtW8G16) {
-                // 32 bytes per row: two uint4, words 0..3 = group 2h, 4..7 = group 2h+1
-                uint4 c0[RW], c1[RW];
-                float s0[RW], s1[RW];
-#pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    const int rr = rbase + r;
-                    if (rr < rows) {
-                        const uint8_t* rowp = st + (size_t)rr * p.crb + (size_t)h * 32;
-                        c0[r] = lds128(rowp);
-                        c1[r] = lds128(rowp + 16);
-                        const uint32_t sp = *reinterpret_cast<const uint32_t*>(ssc + (size_t)rr * p.srb + (size_t)h * 4);
-                        s0[r] = __half2float(__ushort_as_half((unsigned short)(sp & 0xffffu)));
-                        s1[r] = __half2float(__ushort_as_half((unsigned short)(sp >> 16)));
-                    } else {
-                        c0[r] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
-                        c1[r] = c0[r];
-                        s0[r] = s1[r] = 0.0f;
-                    }
-                }
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    float acc[RW][MT];
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float4 xv[MT];
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) xv[m] = xq[((size_t)m * 8 + g * 4 + i) * hcpr];
-#pragma unroll
-                        for (int r = 0; r < RW; ++r) {
-                            const uint4 c = g ? c1[r] : c0[r];
-                            const uint32_t wd = i == 0 ? c.x : i == 1 ? c.y : i == 2 ? c.z : c.w;
-                            float f[4];
-                            unpack_w8(wd, f);
-#pragma unroll
-                            for (int m = 0; m < MT; ++m) {
-                                acc[r][m] = fmaf(f[0], xv[m].x, acc[r][m]);
-                                acc[r][m] = fmaf(f[1], xv[m].y, acc[r][m]);
-                                acc[r][m] = fmaf(f[2], xv[m].z, acc[r][m]);
-                                acc[r][m] = fmaf(f[3], xv[m].w, acc[r][m]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) yacc[r][m] = fmaf(g ? s1[r] : s0[r], acc[r][m], yacc[r][m]);
-                }
-            } else {
-                // int4: 16 bytes (32 nibbles) per row and half-chunk
-                uint4 c[RW];
-                float sA[RW], sB[RW];   // W4G64: (scale, -136 offset); SB32: (S, M)
-#pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    const int rr = rbase + r;
-                    if (rr < rows) {
-                        if (FMT == kFmtW4G64) {
-                            c[r] = lds128(st + (size_t)rr * p.crb + (size_t)h * 16);
-                            const uint16_t sc = *reinterpret_cast<const uint16_t*>(ssc + (size_t)rr * p.srb + (size_t)(h >> 1) * 2);
-                            sA[r] = __half2float(__ushort_as_half(sc));
-                            sB[r] = 0.0f;
-                        } else {
-                            const uint8_t* rec = st + (size_t)rr * p.crb + (size_t)(h >> 3) * 144;
-                            const uint4 hd = lds128(rec);
-                            c[r] = lds128(rec + 16 + (h & 7) * 16);
-                            const int j = h & 7;
-                            const float d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xffffu)));
-                            const float dm = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
-                            sA[r] = __fmul_rn(d, (float)sb_field(hd.y, hd.z, hd.w, 0, j));
-                            sB[r] = __fmul_rn(dm, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
-                        }
-                    } else {
-                        c[r] = make_uint4(0u, 0u, 0u, 0u);
-                        sA[r] = sB[r] = 0.0f;
-                    }
-                }
-                float acc[RW][MT];
-#pragma unroll
-                for (int r = 0; r < RW; ++r)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float4 xa[MT], xb[MT];
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        xa[m] = xq[((size_t)m * 8 + 2 * i) * hcpr];
-                        xb[m] = xq[((size_t)m * 8 + 2 * i + 1) * hcpr];
-                    }
-#pragma unroll
-                    for (int r = 0; r < RW; ++r) {
-                        const uint32_t wd = i == 0 ? c[r].x : i == 1 ? c[r].y : i == 2 ? c[r].z : c[r].w;
-                        float f[8];
-                        unpack_w4(wd, f);
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            float a = acc[r][m];
-                            a = fmaf(f[0], xa[m].x, a);
-                            a = fmaf(f[1], xa[m].y, a);
-                            a = fmaf(f[2], xa[m].z, a);
-                            a = fmaf(f[3], xa[m].w, a);
-                            a = fmaf(f[4], xb[m].x, a);
-                            a = fmaf(f[5], xb[m].y, a);
-                            a = fmaf(f[6], xb[m].z, a);
-                            a = fmaf(f[7], xb[m].w, a);
-                            acc[r][m] = a;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int r = 0; r < RW; ++r)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        if (FMT == kFmtW4G64) {
-                            // s * (sum (128+u) x - 136 sum x) = s * sum q x
-                            yacc[r][m] = fmaf(sA[r], fmaf(-136.0f, xsm[m], acc[r][m]), yacc[r][m]);
-                        } else {
-                            // S * (sum (128+q) x - 128 sum x) - M sum x
-                            yacc[r][m] = fmaf(sA[r], fmaf(-128.0f, xsm[m], acc[r][m]), yacc[r][m]);
-                            yacc[r][m] = fmaf(-sB[r], xsm[m], yacc[r][m]);
-                        }
-                    }
-            }
-        }
-        // stage consumed: release it to the producer
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-
-        // team reduction and store
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                float v = yacc[r][m];
-                for (int o = T >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                yacc[r][m] = v;
-            }
-        if (li == 0) {
-#pragma unroll
-            for (int r = 0; r < RW; ++r) {
-                const int rr = rbase + r;
-                if (rr < rows)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        if (m < p.mrows) p.y[(size_t)(p.m0 + m) * p.N + n0 + rr] = yacc[r][m];
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);       // stage consumed
         }
     }
-    (void)ok;
+    RQ_PHASE_MARK(4);
 }
 
-template <int FMT, int MT, int RW>
-cudaError_t launch_one(const GemvParams& prm, size_t smem, int grid, cudaStream_t st) {
-    auto kern = gemv_kernel<FMT, MT, RW>;
+// Shared-memory target per CTA for single products: three CTAs (three kernels
+// of a dependent chain) fit on one SM. Batches run two CTAs per SM.
+#ifndef RQ_GEMV_SINGLE_CTAS_PER_SM
+#define RQ_GEMV_SINGLE_CTAS_PER_SM 1
+#endif
+#ifndef RQ_GEMV_BATCH_CTAS_PER_SM
+#define RQ_GEMV_BATCH_CTAS_PER_SM 2
+#endif
+constexpr size_t kSmemTarget = 72 * 1024;
+constexpr size_t kSmemBatch = 100 * 1024;
+constexpr size_t kSmemLimit = 220 * 1024;
+constexpr size_t kSmemAttr = kSmemLimit + 1024;
+
+template <int FMT, int MT, int MAXI>
+cudaError_t launch_one(const Batch<MAXI>& prm, size_t smem, int grid, cudaStream_t st) {
+    auto kern = gemv_kernel<FMT, MT, MAXI>;
     // The attribute is per device; set it once per device (a race between
     // host threads only repeats the same idempotent call).
     static unsigned long long attr_done = 0ull;
@@ -317,13 +408,13 @@ cudaError_t launch_one(const GemvParams& prm, size_t smem, int grid, cudaStream_
     if (e != cudaSuccess) return e;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAttr);
         if (e != cudaSuccess) return e;
         __atomic_fetch_or(&attr_done, bit, __ATOMIC_RELEASE);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kGemvThreads);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -334,21 +425,110 @@ cudaError_t launch_one(const GemvParams& prm, size_t smem, int grid, cudaStream_
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
-template <int FMT, int MT>
-cudaError_t launch_rw(const GemvParams& prm, size_t smem, int grid, cudaStream_t st) {
-    return prm.RW == 2 ? launch_one<FMT, MT, 2>(prm, smem, grid, st) : launch_one<FMT, MT, 1>(prm, smem, grid, st);
+// Rows per team allowed for a product: two when a group of 2 * teams rows
+// stays small, else one.
+int rw_allowed(int fmt, int K) {
+    const int hcpr = K / 32;
+    int T = 32;
+    while (T > 1 && (hcpr % T) != 0) T >>= 1;
+    const int teams = kConsumerWarps * (32 / T);
+    auto sb = [&](size_t R) { return round16(R * code_row_bytes(fmt, K)) + round16(R * scale_row_bytes(fmt, K)); };
+    if (sb((size_t)teams * 4) <= 40 * 1024) return 4;
+    return sb((size_t)teams * 2) <= 24 * 1024 ? 2 : 1;
+}
+
+// Per-item launch geometry for rows-per-team RW; false for a shape that does
+// not fit.
+bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b, size_t& x_b) {
+    const bool w4 = fmt != kFmtW8G16;
+    const int hcpr = K / 32;
+    int T = 32;
+    while (T > 1 && (hcpr % T) != 0) T >>= 1;
+    const int teams = kConsumerWarps * (32 / T);
+    const size_t crb = code_row_bytes(fmt, K), srb = scale_row_bytes(fmt, K);
+    int rho = 1;
+    while (((size_t)rho * srb) % 16 != 0) rho <<= 1;     // srb is even, so rho <= 8
+    auto stage_bytes = [&](int R) { return round16((size_t)R * crb) + round16((size_t)R * srb); };
+    x_b = (size_t)MT * K * (w4 ? 2 : 4) + (size_t)MT * hcpr * 4;
+    int Rg = teams * RW;                                 // a power of two >= 8, so a multiple of rho
+    while (Rg > rho && Rg > RW && x_b + 2 * stage_bytes(Rg) + 64 > kSmemLimit) Rg >>= 1;
+    if (x_b + stage_bytes(Rg) + 64 > kSmemLimit) return false;
+    it.K = K;
+    it.N = N;
+    it.T = T;
+    it.HJ = hcpr / T;
+    it.RW = RW;
+    it.Rg = Rg;
+    it.rho = rho;
+    it.crb = (uint32_t)crb;
+    it.srb = (uint32_t)srb;
+    it.ucost = (uint32_t)((size_t)rho * (crb + srb));
+    stage_b = stage_bytes(Rg);
+    return true;
+}
+
+template <int FMT, int MAXI>
+cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
+    const int M = a[0].M;
+    const int MT = M >= 2 ? 2 : 1;
+    Batch<MAXI> p = {};
+    p.count = count;
+    size_t sb = 0, xq = 0, xs = 0;
+    long long total = 0, units_min = -1;
+    for (int i = 0; i < count; ++i) {
+        Item& it = p.it[i];
+        size_t s1, x1;
+        if (!plan_item(FMT, a[i].K, a[i].N, MT, rw_allowed(FMT, a[i].K), it, s1, x1)) return cudaErrorInvalidValue;
+        it.x = static_cast<const uint16_t*>(a[i].x);
+        it.codes = static_cast<const uint8_t*>(a[i].codes);
+        it.scales = static_cast<const uint8_t*>(a[i].scales);
+        it.y = a[i].y;
+        it.cost0 = total;
+        const long long U = (it.N + it.rho - 1) / it.rho;
+        total += U * it.ucost;
+        units_min = units_min < 0 || U < units_min ? U : units_min;
+        sb = s1 > sb ? s1 : sb;
+        const size_t q = (size_t)MT * a[i].K * (FMT != kFmtW8G16 ? 2 : 4), s = (size_t)MT * (a[i].K / 32) * 4;
+        xq = q > xq ? q : xq;
+        xs = s > xs ? s : xs;
+    }
+    p.total = total;
+    int grid = sm_count() * (count > 1 ? RQ_GEMV_BATCH_CTAS_PER_SM : RQ_GEMV_SINGLE_CTAS_PER_SM);
+    if (count == 1 && grid > units_min) grid = (int)units_min;
+    const size_t fixed = xq + xs + 64;
+    const size_t want = count > 1 ? kSmemBatch : kSmemTarget;
+    const size_t budget = fixed + 2 * sb <= want ? want : kSmemLimit;
+    int stages = (int)((budget - fixed) / sb);
+    if (stages > 6) stages = 6;
+    if (count == 1) {   // a single product needs no more stages than its largest CTA has groups
+        const Item& it = p.it[0];
+        const long long per = (units_min + grid - 1) / grid * it.rho;
+        const int gmax = (int)((per + it.Rg - 1) / it.Rg);
+        if (stages > gmax) stages = gmax;
+    }
+    if (stages < 1) return cudaErrorInvalidValue;
+    p.stages = stages;
+    p.stage_bytes = (uint32_t)sb;
+    p.x_off = (uint32_t)(stages * sb);
+    p.xsum_off = (uint32_t)(p.x_off + xq);
+    p.bar_off = (uint32_t)round16(p.xsum_off + xs);
+    const size_t smem = p.bar_off + 2 * stages * sizeof(uint64_t);
+    if (smem > kSmemAttr) return cudaErrorInvalidValue;
+
+    for (int m0 = 0; m0 < M; m0 += MT) {
+        p.m0 = m0;
+        p.mrows = M - m0 < MT ? M - m0 : MT;
+        const cudaError_t e = MT == 2 ? launch_one<FMT, 2, MAXI>(p, smem, grid, st)
+                                      : launch_one<FMT, 1, MAXI>(p, smem, grid, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 template <int FMT>
-cudaError_t launch_mt(int MT, const GemvParams& prm, size_t smem, int grid, cudaStream_t st) {
-    switch (MT) {
-        case 4: return launch_rw<FMT, 4>(prm, smem, grid, st);
-        case 2: return launch_rw<FMT, 2>(prm, smem, grid, st);
-        default: return launch_rw<FMT, 1>(prm, smem, grid, st);
-    }
+cudaError_t launch_fmt(const WgemmArgs* a, int count, cudaStream_t st) {
+    return count == 1 ? launch_batch<FMT, 1>(a, count, st) : launch_batch<FMT, kMaxBatch>(a, count, st);
 }
-
-constexpr size_t kSmemBudget = 220 * 1024;
 
 }  // namespace
 
@@ -361,67 +541,12 @@ cudaError_t status_gemv(cudaStream_t st, unsigned* word) {
     return e;
 }
 
-cudaError_t launch_gemv(const WgemmArgs& a, cudaStream_t st) {
-    const int K = a.K, N = a.N;
-    const int hcpr = K / 32;
-    int T = 32;
-    while (T > 1 && (hcpr % T) != 0) T >>= 1;
-    const int teams = kConsumerWarps * (32 / T);
-    const size_t crb = code_row_bytes(a.fmt, K), srb = scale_row_bytes(a.fmt, K);
-
-    auto stage_bytes = [&](int R) { return round16((size_t)R * crb) + round16((size_t)R * srb); };
-    const int RW = stage_bytes(teams * 2) <= 24 * 1024 ? 2 : 1;
-    const int R = teams * RW;
-    const size_t sb = stage_bytes(R);
-
-    int MT = a.M >= 4 ? 4 : (a.M >= 2 ? 2 : 1);
-    auto x_bytes = [&](int mt) { return (size_t)mt * K * 4 + (size_t)mt * hcpr * 4; };
-    while (MT > 1 && x_bytes(MT) + 2 * sb > kSmemBudget) MT >>= 1;
-    const size_t xb = x_bytes(MT);
-    if (xb + 2 * sb + 64 > kSmemBudget) return cudaErrorInvalidValue;
-    int stages = (int)((kSmemBudget - xb - 64) / sb);
-    stages = stages > 4 ? 4 : stages;
-
-    GemvParams p = {};
-    p.x = static_cast<const uint16_t*>(a.x);
-    p.codes = static_cast<const uint8_t*>(a.codes);
-    p.scales = static_cast<const uint8_t*>(a.scales);
-    p.y = a.y;
-    p.K = K;
-    p.N = N;
-    p.T = T;
-    p.HJ = hcpr / T;
-    p.RW = RW;
-    p.R = R;
-    p.stages = stages;
-    p.tiles = (N + R - 1) / R;
-    p.crb = (uint32_t)crb;
-    p.srb = (uint32_t)srb;
-    p.stage_bytes = (uint32_t)sb;
-    p.scale_off = (uint32_t)round16((size_t)R * crb);
-    p.x_off = (uint32_t)(stages * sb);
-    p.bar_off = (uint32_t)(p.x_off + xb);
-    const size_t smem = p.bar_off + 2 * stages * sizeof(uint64_t);
-
-    // CTAs resident per SM for this footprint (smem and threads), then one
-    // wave of CTAs that loop over the tiles.
-    int per_sm = (int)(228 * 1024 / (smem + 1024));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 2048 / kGemvThreads ? 2048 / kGemvThreads : per_sm);
-    int grid = sm_count() * per_sm;
-    if (grid > p.tiles) grid = p.tiles;
-
-    for (int m0 = 0; m0 < a.M; m0 += MT) {
-        p.m0 = m0;
-        p.mrows = a.M - m0 < MT ? a.M - m0 : MT;
-        cudaError_t e;
-        switch (a.fmt) {
-            case kFmtW4G64: e = launch_mt<kFmtW4G64>(MT, p, smem, grid, st); break;
-            case kFmtW8G16: e = launch_mt<kFmtW8G16>(MT, p, smem, grid, st); break;
-            default: e = launch_mt<kFmtW4SB32>(MT, p, smem, grid, st); break;
-        }
-        if (e != cudaSuccess) return e;
+cudaError_t launch_gemv(const WgemmArgs* a, int count, cudaStream_t st) {
+    switch (a[0].fmt) {
+        case kFmtW4G64: return launch_fmt<kFmtW4G64>(a, count, st);
+        case kFmtW8G16: return launch_fmt<kFmtW8G16>(a, count, st);
+        default: return launch_fmt<kFmtW4SB32>(a, count, st);
     }
-    return cudaSuccess;
 }
 
 }  // namespace rq

@@ -20,7 +20,7 @@ inline size_t code_row_bytes(int fmt, int K) {
 inline size_t scale_row_bytes(int fmt, int K) {
     return fmt == kFmtW4G64 ? (size_t)K / 32 : fmt == kFmtW8G16 ? (size_t)K / 8 : 0;
 }
-inline size_t round16(size_t v) { return (v + 15) & ~(size_t)15; }
+__host__ __device__ inline size_t round16(size_t v) { return (v + 15) & ~(size_t)15; }
 
 struct PackArgs {
     int fmt, K, N;
@@ -45,8 +45,11 @@ struct WgemmArgs {
     float* y;              // fp32 [M][N]
 };
 
-// Memory-bound path (few activation rows): dequantize in registers, fp32 FMA.
-cudaError_t launch_gemv(const WgemmArgs& a, cudaStream_t st);
+// Memory-bound path (few activation rows): dequantize in registers, fp32
+// accumulate. `count` independent products of one format and one M share a
+// launch (1 <= count <= kMaxBatch).
+constexpr int kMaxBatch = 160;
+cudaError_t launch_gemv(const WgemmArgs* a, int count, cudaStream_t st);
 
 // Read and clear the device status word of each kernel file (synchronizes st).
 cudaError_t status_pack(cudaStream_t st, unsigned* word);

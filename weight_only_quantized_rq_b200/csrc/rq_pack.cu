@@ -259,10 +259,10 @@ __global__ void dequant_w4_kernel(const uint32_t* __restrict__ codes, const __ha
     const long long n = i / wpr;
     const int k0 = (int)(i % wpr) * 8;
     const float s = __half2float(scales[n * (K / 64) + k0 / 64]);
-    float f[8], o[8];
-    unpack_w4(codes[i], f);
+    float o[8];
+    w4_word_values(codes[i], o);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) o[w4_slot_nibble(j)] = __fmul_rn(__fsub_rn(f[j], 136.0f), s);
+    for (int j = 0; j < 8; ++j) o[j] = __fmul_rn(__fsub_rn(o[j], 136.0f), s);
     float4* dst = reinterpret_cast<float4*>(out + n * K + k0);
     dst[0] = make_float4(o[0], o[1], o[2], o[3]);
     dst[1] = make_float4(o[4], o[5], o[6], o[7]);
@@ -299,10 +299,10 @@ __global__ void dequant_sb32_kernel(const uint8_t* __restrict__ blocks, int K, l
     const int j = wi / 4;   // 4 words (32 weights) per group
     const float S = __fmul_rn(d, (float)sb_field(r[1], r[2], r[3], 0, j));
     const float M = __fmul_rn(dm, (float)sb_field(r[1], r[2], r[3], 1, j));
-    float f[8], o[8];
-    unpack_w4(r[4 + wi], f);
+    float o[8];
+    w4_word_values(r[4 + wi], o);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) o[w4_slot_nibble(s)] = __fmaf_rn(S, __fsub_rn(f[s], 128.0f), -M);
+    for (int s = 0; s < 8; ++s) o[s] = __fmaf_rn(S, __fsub_rn(o[s], 128.0f), -M);
     float4* dst = reinterpret_cast<float4*>(out + n * K + (size_t)b * 256 + wi * 8);
     dst[0] = make_float4(o[0], o[1], o[2], o[3]);
     dst[1] = make_float4(o[4], o[5], o[6], o[7]);

@@ -56,8 +56,10 @@ struct Item {                  // one product of a launch
     const uint8_t* scales;
     float* y;                  // fp32 [M][N]
     long long cost0;           // packed bytes of the items before this one
+    long long cost1;           // cost0 + this item's packed bytes
     int K, N;
-    int T, HJ;                 // team lanes, half-chunks per lane
+    int T, HJ;                 // team lanes, half-chunks per lane and warp
+    int KS;                    // warps sharing a row (each takes HJ * T consecutive half-chunk slots)
     int RW, Rg;                // rows per team, rows per group (a multiple of rho)
     int rho;                   // rows per unit; a unit is the grain of the CTA split
     uint32_t crb, srb;         // code / scale bytes per row
@@ -69,7 +71,7 @@ struct Batch {
     int count, m0, mrows;      // items; activation rows [m0, m0 + mrows) of every item
     int stages;
     long long total;           // packed bytes of all items
-    uint32_t stage_bytes, x_off, xsum_off, bar_off;
+    uint32_t stage_bytes, x_off, xsum_off, red_off, red_bytes, bar_off;
     Item it[MAXI];
 };
 
@@ -131,11 +133,13 @@ __device__ __forceinline__ uint32_t word_of(const uint4& c, int i) {
 // stored.
 template <int FMT, int MT, int RW>
 __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s,
-                                           uint32_t xsum_s, int m0, int mrows, int lane, int rbase) {
+                                           uint32_t xsum_s, int m0, int mrows, int lane, int rbase, int slice,
+                                           float* red) {
     constexpr bool kW4 = FMT != kFmtW8G16;
     constexpr int U = RW == 1 ? 2 : 1;                   // half-chunks per iteration
     const int hcpr = it.K >> 5, T = it.T, HJ = it.HJ;
     const int li = lane & (T - 1);
+    const int hoff = slice * HJ;                         // this warp's k-slice of the row
     const uint32_t crb = it.crb, srb = it.srb;
     const uint32_t ssc_s = st_s + (uint32_t)round16((size_t)it.Rg * crb);
     // x quads: (m * Q + q) * hcpr + h, Q = 4 (bf16) or 8 (fp32) quads per half-chunk
@@ -171,7 +175,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (u > 0 && hj + u >= HJ) break;
-                const uint32_t dh = (uint32_t)(hj + u) * (uint32_t)T;
+                const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
                 float xsm[MT];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) xsm[m] = ldsf_a(xs0 + (uint32_t)m * (uint32_t)hcpr * 4u + dh * 4u);
@@ -236,7 +240,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (u > 0 && hj + u >= HJ) break;
-                const uint32_t dh = (uint32_t)(hj + u) * (uint32_t)T;
+                const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
 #pragma unroll
                 for (int r = 0; r < RW; ++r) {
                     const uint4 c0 = lds128_a(ca[r] + dh * 32u);
@@ -269,6 +273,33 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             }
         }
     }
+    if (T == 32 && RW == 4) {
+        // Recursive halving over the warp: after the offset-16 step lanes 0-15
+        // hold rows {0,1} and lanes 16-31 rows {2,3}; after offset 8 each lane
+        // holds one row (lane bits 4..3); three more steps finish the sum, so
+        // lane 8r holds row r.
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const bool up16 = (lane & 16) != 0;
+            float a0 = up16 ? yacc[2 % RW][m] : yacc[0][m], a1 = up16 ? yacc[3 % RW][m] : yacc[1 % RW][m];
+            const float give0 = up16 ? yacc[0][m] : yacc[2 % RW][m], give1 = up16 ? yacc[1 % RW][m] : yacc[3 % RW][m];
+            a0 += __shfl_xor_sync(0xffffffffu, give0, 16);
+            a1 += __shfl_xor_sync(0xffffffffu, give1, 16);
+            const bool up8 = (lane & 8) != 0;
+            float v = up8 ? a1 : a0;
+            v += __shfl_xor_sync(0xffffffffu, up8 ? a0 : a1, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            const int r = lane >> 3;                     // row of this lane's sum
+            const int rr = rbase + r;
+            if ((lane & 7) == 0 && rr < rg) {
+                if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = v;
+                else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = v;
+            }
+        }
+        return;
+    }
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
@@ -283,8 +314,10 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             const int rr = rbase + r;
             if (rr < rg)
 #pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = yacc[r][m];
+                for (int m = 0; m < MT; ++m) {
+                    if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = yacc[r][m];
+                    else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = yacc[r][m];
+                }
         }
     }
 }
@@ -319,6 +352,8 @@ gemv_kernel(const Batch<MAXI> p) {
             bool ok = true;
             for (int i = 0; i < p.count && ok; ++i) {
                 const Item& it = p.it[i];
+                if (it.cost0 >= hi) break;               // items are in cost order
+                if (it.cost1 <= lo) continue;            // no overlap: skip without dividing
                 int ua, ub;
                 item_units(it, lo, hi, ua, ub);
                 const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
@@ -350,6 +385,8 @@ gemv_kernel(const Batch<MAXI> p) {
     bool first = true;
     for (int i = 0; i < p.count; ++i) {
         const Item& it = p.it[i];
+        if (it.cost0 >= hi) break;                       // items are in cost order
+        if (it.cost1 <= lo) continue;                    // no overlap: skip without dividing
         int ua, ub;
         item_units(it, lo, hi, ua, ub);
         const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
@@ -359,26 +396,40 @@ gemv_kernel(const Batch<MAXI> p) {
         stage_x<FMT, MT>(it, p.m0, p.mrows, xbuf, xsum, tid);
         asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
         RQ_PHASE_MARK(2);
-        const int T = it.T, RW = it.RW;
-        const int team = lane / T;
-        const int rbase = (warp * (32 / T) + team) * RW;      // first row of this team in a group
-        const int wfirst = warp * (32 / T) * RW;               // first row of this warp in a group
+        const int T = it.T, RW = it.RW, KS = it.KS;
+        const int slice = warp % KS;                     // k-slice of this warp (KS > 1 only when T == 32)
+        const int wteam = (warp / KS) * (32 / T);         // first team of this warp
+        const int rbase = (wteam + lane / T) * RW;        // first row of this team in a group
+        const int wfirst = wteam * RW;                    // first row of this warp in a group
         for (int g0 = ra; g0 < rb; g0 += it.Rg, ++gi) {
             const int s = gi % p.stages;
             if (!mbar_wait_bounded(&full[s], (gi / p.stages) & 1, kStatusTmaWait)) return;
             RQ_PHASE_MARK(3);
             const int rg = min(it.Rg, rb - g0);
+            float* red = reinterpret_cast<float*>(smem + p.red_off + (gi & 1) * p.red_bytes);
             if (wfirst < rg) {                           // warp-uniform
                 const uint32_t st_s = smem_s + (uint32_t)s * p.stage_bytes;
                 if (RW == 4)
-                    gemv_group<FMT, MT, 4>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows, lane, rbase);
+                    gemv_group<FMT, MT, 4>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows,
+                                           lane, rbase, slice, red);
                 else if (RW == 2)
-                    gemv_group<FMT, MT, 2>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows, lane, rbase);
+                    gemv_group<FMT, MT, 2>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows,
+                                           lane, rbase, slice, red);
                 else
-                    gemv_group<FMT, MT, 1>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows, lane, rbase);
+                    gemv_group<FMT, MT, 1>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows,
+                                           lane, rbase, slice, red);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);       // stage consumed
+            if (KS > 1) {                                // combine the k-slices of each row
+                asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
+                for (int t = tid; t < rg * MT; t += kConsumerWarps * 32) {
+                    const int rr = t / MT, m = t - rr * MT;
+                    float v = 0.0f;
+                    for (int k = 0; k < KS; ++k) v += red[(size_t)t * KS + k];
+                    if (m < p.mrows) it.y[(size_t)(p.m0 + m) * it.N + g0 + rr] = v;
+                }
+            }
         }
     }
     RQ_PHASE_MARK(4);
@@ -425,16 +476,30 @@ cudaError_t launch_one(const Batch<MAXI>& prm, size_t smem, int grid, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
-// Rows per team allowed for a product: two when a group of 2 * teams rows
-// stays small, else one.
-int rw_allowed(int fmt, int K) {
+// Lane and warp layout of a product's rows: T lanes per team (a power of two
+// dividing K/32), KS warps per row (when T == 32, long rows are split so that
+// each warp covers about two half-chunks per lane), HJ half-chunks per lane.
+struct Layout { int T, KS, HJ, teams; };
+Layout layout_of(int K) {
     const int hcpr = K / 32;
-    int T = 32;
-    while (T > 1 && (hcpr % T) != 0) T >>= 1;
-    const int teams = kConsumerWarps * (32 / T);
+    Layout l;
+    l.T = 32;
+    while (l.T > 1 && (hcpr % l.T) != 0) l.T >>= 1;
+    const int hj_all = hcpr / l.T;
+    l.KS = 1;
+    while (l.T == 32 && l.KS * 2 <= kConsumerWarps && hj_all % (l.KS * 2) == 0 && hj_all / (l.KS * 2) >= 2) l.KS *= 2;
+    l.HJ = hj_all / l.KS;
+    l.teams = (kConsumerWarps / l.KS) * (32 / l.T);
+    return l;
+}
+
+// Rows per team for a product: the largest of 4, 2, 1 whose group of
+// teams * RW rows stays within 48 KB.
+int rw_allowed(int fmt, int K) {
+    const Layout l = layout_of(K);
     auto sb = [&](size_t R) { return round16(R * code_row_bytes(fmt, K)) + round16(R * scale_row_bytes(fmt, K)); };
-    if (sb((size_t)teams * 4) <= 40 * 1024) return 4;
-    return sb((size_t)teams * 2) <= 24 * 1024 ? 2 : 1;
+    if (sb((size_t)l.teams * 4) <= 48 * 1024) return 4;
+    return sb((size_t)l.teams * 2) <= 48 * 1024 ? 2 : 1;
 }
 
 // Per-item launch geometry for rows-per-team RW; false for a shape that does
@@ -442,21 +507,20 @@ int rw_allowed(int fmt, int K) {
 bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b, size_t& x_b) {
     const bool w4 = fmt != kFmtW8G16;
     const int hcpr = K / 32;
-    int T = 32;
-    while (T > 1 && (hcpr % T) != 0) T >>= 1;
-    const int teams = kConsumerWarps * (32 / T);
+    const Layout l = layout_of(K);
     const size_t crb = code_row_bytes(fmt, K), srb = scale_row_bytes(fmt, K);
     int rho = 1;
     while (((size_t)rho * srb) % 16 != 0) rho <<= 1;     // srb is even, so rho <= 8
     auto stage_bytes = [&](int R) { return round16((size_t)R * crb) + round16((size_t)R * srb); };
     x_b = (size_t)MT * K * (w4 ? 2 : 4) + (size_t)MT * hcpr * 4;
-    int Rg = teams * RW;                                 // a power of two >= 8, so a multiple of rho
+    int Rg = l.teams * RW;                               // a power of two
     while (Rg > rho && Rg > RW && x_b + 2 * stage_bytes(Rg) + 64 > kSmemLimit) Rg >>= 1;
-    if (x_b + stage_bytes(Rg) + 64 > kSmemLimit) return false;
+    if (Rg % rho != 0 || x_b + stage_bytes(Rg) + 64 > kSmemLimit) return false;
     it.K = K;
     it.N = N;
-    it.T = T;
-    it.HJ = hcpr / T;
+    it.T = l.T;
+    it.HJ = l.HJ;
+    it.KS = l.KS;
     it.RW = RW;
     it.Rg = Rg;
     it.rho = rho;
@@ -473,7 +537,7 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
     const int MT = M >= 2 ? 2 : 1;
     Batch<MAXI> p = {};
     p.count = count;
-    size_t sb = 0, xq = 0, xs = 0;
+    size_t sb = 0, xq = 0, xs = 0, red = 0;
     long long total = 0, units_min = -1;
     for (int i = 0; i < count; ++i) {
         Item& it = p.it[i];
@@ -486,16 +550,19 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
         it.cost0 = total;
         const long long U = (it.N + it.rho - 1) / it.rho;
         total += U * it.ucost;
+        it.cost1 = total;
         units_min = units_min < 0 || U < units_min ? U : units_min;
         sb = s1 > sb ? s1 : sb;
         const size_t q = (size_t)MT * a[i].K * (FMT != kFmtW8G16 ? 2 : 4), s = (size_t)MT * (a[i].K / 32) * 4;
         xq = q > xq ? q : xq;
         xs = s > xs ? s : xs;
+        const size_t rd = it.KS > 1 ? round16((size_t)it.Rg * MT * it.KS * 4) : 0;
+        red = rd > red ? rd : red;
     }
     p.total = total;
     int grid = sm_count() * (count > 1 ? RQ_GEMV_BATCH_CTAS_PER_SM : RQ_GEMV_SINGLE_CTAS_PER_SM);
     if (count == 1 && grid > units_min) grid = (int)units_min;
-    const size_t fixed = xq + xs + 64;
+    const size_t fixed = xq + xs + 2 * red + 64;
     const size_t want = count > 1 ? kSmemBatch : kSmemTarget;
     const size_t budget = fixed + 2 * sb <= want ? want : kSmemLimit;
     int stages = (int)((budget - fixed) / sb);
@@ -511,7 +578,9 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
     p.stage_bytes = (uint32_t)sb;
     p.x_off = (uint32_t)(stages * sb);
     p.xsum_off = (uint32_t)(p.x_off + xq);
-    p.bar_off = (uint32_t)round16(p.xsum_off + xs);
+    p.red_off = (uint32_t)round16(p.xsum_off + xs);
+    p.red_bytes = (uint32_t)red;
+    p.bar_off = (uint32_t)round16(p.red_off + 2 * red);
     const size_t smem = p.bar_off + 2 * stages * sizeof(uint64_t);
     if (smem > kSmemAttr) return cudaErrorInvalidValue;
 

@@ -276,6 +276,57 @@ __device__ __forceinline__ float dot8_w4(uint32_t w, uint4 X, float acc) {
     return acc;
 }
 
+// int4 codes as fp16 pairs (the GEMV unpack). An fp16 mantissa has ten bits,
+// so both nibbles of a byte fit under the exponent pattern 0x64 (fp16 1024.0,
+// mantissa bit 0 weighs 1): masking nibble positions 0 and 4 of each 16-bit
+// half gives (1024 + u), positions 1 and 5 give (1024 + 16 u). Pairs of word
+// w: P0 = (k0, k4), P1 = (k1, k5) from w; P2 = (k2, k6), P3 = (k3, k7) from
+// w >> 8. One shift and four three-input logic ops per eight weights.
+constexpr uint32_t kW4HalfMagic = 0x64006400u;
+
+__device__ __forceinline__ uint32_t lop_or_mask(uint32_t v, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(v), "r"(m), "r"(kW4HalfMagic));  // (v & m) | c
+    return d;
+}
+
+// c + a.half(AH) * b.half(BH) with fp16 operands and an fp32 accumulator; the
+// product of two fp16 values is exact in fp32 (one rounding, in the add).
+template <int AH, int BH>
+__device__ __forceinline__ float fma_f16(uint32_t a, uint32_t b, float c) {
+    float d;
+    if (AH == 0 && BH == 0)
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.f16 %0, a0, b0, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if (AH == 1 && BH == 0)
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.f16 %0, a1, b0, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if (AH == 0 && BH == 1)
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.f16 %0, a0, b1, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else
+        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
+            " fma.rn.f32.f16 %0, a1, b1, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+// One code word against x_0..x_7 (fp16, natural-order pairs X.x = (x0, x1),
+// X.y = (x2, x3), X.z = (x4, x5), X.w = (x6, x7)): even k go to lo0/lo1 as
+// (1024 + u_k) x_k, odd k to hi0/hi1 as (1024 + 16 u_k) x_k.
+__device__ __forceinline__ void dot8_w4_f16(uint32_t w, uint4 X, float& lo0, float& lo1, float& hi0, float& hi1) {
+    const uint32_t v = w >> 8;
+    const uint32_t p0 = lop_or_mask(w, 0x000F000Fu), p1 = lop_or_mask(w, 0x00F000F0u);
+    const uint32_t p2 = lop_or_mask(v, 0x000F000Fu), p3 = lop_or_mask(v, 0x00F000F0u);
+    lo0 = fma_f16<0, 0>(p0, X.x, lo0);   // k0
+    lo1 = fma_f16<1, 0>(p0, X.z, lo1);   // k4
+    hi0 = fma_f16<0, 1>(p1, X.x, hi0);   // k1
+    hi1 = fma_f16<1, 1>(p1, X.z, hi1);   // k5
+    lo0 = fma_f16<0, 0>(p2, X.y, lo0);   // k2
+    lo1 = fma_f16<1, 0>(p2, X.w, lo1);   // k6
+    hi0 = fma_f16<0, 1>(p3, X.y, hi0);   // k3
+    hi1 = fma_f16<1, 1>(p3, X.w, hi1);   // k7
+}
+
 // int8 codes. Byte k of a word is the code u = q + 128 of weight k. Each byte
 // is placed in bits 8..15 under exponent byte 0x47 (fp32 32768.0, mantissa
 // bit 8 weighs 1), giving 32768 + u; subtracting 32896 gives q exactly.

@@ -20,13 +20,16 @@
 //    stream in while the previous kernel finishes.
 //  * After the wait, each product's x is staged in shared memory, interleaved
 //    by 16-byte quads so that lanes reading consecutive half-chunks (32
-//    weights) hit consecutive banks, with the sum of x over each half-chunk.
+//    weights) hit consecutive banks. For int4, x is held as fp16 under a
+//    power-of-two scale per half-chunk, with the half-chunk's offset sums.
 //  * A team of T lanes (a power of two dividing K/32) owns RW rows of a group;
-//    lane i takes half-chunks i, i+T, ... of those rows.
-//    int4: one shift + one lop3 turns two nibbles into the bf16 pair
-//    (128 + u, 128 + u'), multiplied by bf16 x with fp32-accumulating
-//    fma.rn.f32.bf16; the scale and code offset are applied once per
-//    half-chunk:  sum_k (u_k - 8) x_k s = s (sum_k (128 + u_k) x_k - 136 sum_k x_k).
+//    lane i takes half-chunks i, i+T, ... of those rows; long rows are split
+//    over KS warps whose partial sums meet in shared memory.
+//    int4: a lop3 with mask and exponent pattern turns two nibbles into an
+//    fp16 pair ((1024 + u), or (1024 + 16 u) for the upper nibble of a byte),
+//    one shift and four lop3 per eight weights, multiplied by the fp16 x with
+//    fp32-accumulating fma.rn.f32.f16; scale and code offset are applied once
+//    per half-chunk:  sum_k (u_k - 8) x_k s = s f (lo + hi / 16 - z).
 //    int8: a byte permute places each code under an fp32 exponent (32768 + u),
 //    one subtraction gives q exactly, fp32 fma with fp32 x.
 //  * Team partial sums are reduced with warp shuffles; one store per output.
@@ -71,7 +74,7 @@ struct Batch {
     int count, m0, mrows;      // items; activation rows [m0, m0 + mrows) of every item
     int stages;
     long long total;           // packed bytes of all items
-    uint32_t stage_bytes, x_off, xsum_off, red_off, red_bytes, bar_off;
+    uint32_t stage_bytes, x_off, xmeta_off, red_off, red_bytes, bar_off;
     Item it[MAXI];
 };
 
@@ -88,8 +91,18 @@ __device__ __forceinline__ void item_units(const Item& it, long long lo, long lo
     ub = (int)first_at_or_after(hi);
 }
 
+// Staged x for one product and activation rows [m0, m0 + MT).
+//  int4 formats: fp16 quads in natural order (quad q = x[8q .. 8q+7]), each
+//  half-chunk h (32 values) scaled by its own power of two 2^e_h so that its
+//  largest |x| lies in [2^14, 2^15) (exact for every value that stays a
+//  normal fp16, i.e. all but those 2^28 times smaller than the largest), and
+//  a float4 per half-chunk {z, sx, f, 0}: f = 2^-e_h, sx = sum of the scaled
+//  values, z = the code offsets' share (g64: 1032 * sum over even k + 72 *
+//  sum over odd k; sb32: 1024 / 64), summed from the fp16 values the products
+//  use.
+//  int8 format: fp32 quads (quad q = x[4q .. 4q+3]).
 template <int FMT, int MT>
-__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xbuf, float* xsum, int tid) {
+__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xbuf, float4* xmeta, int tid) {
     constexpr bool kW4 = FMT != kFmtW8G16;
     const int hcpr = it.K >> 5;
     for (int i = tid; i < MT * hcpr; i += kConsumerWarps * 32) {
@@ -100,25 +113,36 @@ __device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8
 #pragma unroll
             for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
         }
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
-        if (kW4) {   // bf16 quads, natural order: quad q = x[8q .. 8q+7]
+        uint32_t* w = reinterpret_cast<uint32_t*>(v);
+        if (kW4) {
+            uint32_t mb = 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
+            int e = 0;
+            if (mb != 0) e = min(126, max(-126, 14 - ((int)(mb >> 7) - 127)));
+            const float up = __int_as_float((e + 127) << 23);
+            float se = 0.0f, so = 0.0f;                  // even-k and odd-k sums
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
+                const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+                se = __fadd_rn(se, __half2float(a));
+                so = __fadd_rn(so, __half2float(b));
+                w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+            }
             uint4* dst = reinterpret_cast<uint4*>(xbuf) + (size_t)m * 4 * hcpr + h;
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[q];
-        } else {     // fp32 quads, natural order: quad q = x[4q .. 4q+3]
+            const float z = FMT == kFmtW4G64 ? __fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so))
+                                             : __fmaf_rn(1024.0f, se, __fmul_rn(64.0f, so));
+            xmeta[(size_t)m * hcpr + h] = make_float4(z, __fadd_rn(se, so), __int_as_float((127 - e) << 23), 0.0f);
+        } else {
             float4* dst = reinterpret_cast<float4*>(xbuf) + (size_t)m * 8 * hcpr + h;
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 dst[(size_t)q * hcpr] = make_float4(bf16lo_f32(w[2 * q]), bf16hi_f32(w[2 * q]),
                                                     bf16lo_f32(w[2 * q + 1]), bf16hi_f32(w[2 * q + 1]));
         }
-        float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-            s0 += bf16lo_f32(w[j]) + bf16hi_f32(w[j]);
-            s1 += bf16lo_f32(w[j + 1]) + bf16hi_f32(w[j + 1]);
-        }
-        xsum[(size_t)m * hcpr + h] = s0 + s1;
     }
 }
 
@@ -133,7 +157,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& c, int i) {
 // stored.
 template <int FMT, int MT, int RW>
 __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s,
-                                           uint32_t xsum_s, int m0, int mrows, int lane, int rbase, int slice,
+                                           uint32_t xmeta_s, int m0, int mrows, int lane, int rbase, int slice,
                                            float* red) {
     constexpr bool kW4 = FMT != kFmtW8G16;
     constexpr int U = RW == 1 ? 2 : 1;                   // half-chunks per iteration
@@ -145,7 +169,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
     // x quads: (m * Q + q) * hcpr + h, Q = 4 (bf16) or 8 (fp32) quads per half-chunk
     const uint32_t xstride = (uint32_t)hcpr * 16u;
     const uint32_t xa0 = x_s + (uint32_t)li * 16u;
-    const uint32_t xs0 = xsum_s + (uint32_t)li * 4u;
+    const uint32_t xm0 = xmeta_s + (uint32_t)li * 16u;
     float yacc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
@@ -168,17 +192,14 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                 sa[r] = 0u;
             }
         }
-        // four accumulators per row and m, whatever the launch shape, so a row's
-        // sums (and results) do not depend on RW or on batching
-        constexpr int NA = 4;
         for (int hj = 0; hj < HJ; hj += U) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (u > 0 && hj + u >= HJ) break;
                 const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
-                float xsm[MT];
+                float4 xm[MT];
 #pragma unroll
-                for (int m = 0; m < MT; ++m) xsm[m] = ldsf_a(xs0 + (uint32_t)m * (uint32_t)hcpr * 4u + dh * 4u);
+                for (int m = 0; m < MT; ++m) xm[m] = lds128f_a(xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * 16u);
                 uint4 c[RW];
                 float sA[RW], sB[RW];
 #pragma unroll
@@ -197,32 +218,37 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                         sB[r] = __fmul_rn(dm, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
                     }
                 }
-                float acc[RW][MT][NA];
+                // two accumulators for even k ((1024 + u) x) and two for odd k
+                // ((1024 + 16 u) x) per row and m, whatever the launch shape, so
+                // a row's sums (and results) do not depend on RW or on batching
+                float lo0[RW][MT], lo1[RW][MT], hi0[RW][MT], hi1[RW][MT];
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
-                    for (int m = 0; m < MT; ++m)
-#pragma unroll
-                        for (int k = 0; k < NA; ++k) acc[r][m][k] = 0.0f;
+                    for (int m = 0; m < MT; ++m) lo0[r][m] = lo1[r][m] = hi0[r][m] = hi1[r][m] = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         const uint4 X = lds128_a(xa0 + dh * 16u + (uint32_t)(m * 4 + i) * xstride);
 #pragma unroll
-                        for (int r = 0; r < RW; ++r) dot8_w4_split<NA>(word_of(c[r], i), X, acc[r][m]);
+                        for (int r = 0; r < RW; ++r)
+                            dot8_w4_f16(word_of(c[r], i), X, lo0[r][m], lo1[r][m], hi0[r][m], hi1[r][m]);
                     }
                 }
+                // sum_k q_k x'_k = lo + hi / 16 - z; scaled back by f = 2^-e_h
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
-                        const float a = sum_acc<NA>(acc[r][m]);
+                        const float a = __fmaf_rn(__fadd_rn(hi0[r][m], hi1[r][m]), 0.0625f,
+                                                  __fadd_rn(lo0[r][m], lo1[r][m]));
+                        const float t = __fsub_rn(a, xm[m].x);
                         if (FMT == kFmtW4G64) {
-                            yacc[r][m] = fmaf(sA[r], fmaf(-136.0f, xsm[m], a), yacc[r][m]);
+                            yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].z), t, yacc[r][m]);
                         } else {
-                            yacc[r][m] = fmaf(sA[r], fmaf(-128.0f, xsm[m], a), yacc[r][m]);
-                            yacc[r][m] = fmaf(-sB[r], xsm[m], yacc[r][m]);
+                            const float v = __fmaf_rn(-sB[r], xm[m].y, __fmul_rn(sA[r], t));
+                            yacc[r][m] = __fmaf_rn(xm[m].z, v, yacc[r][m]);
                         }
                     }
             }
@@ -322,15 +348,20 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
     }
 }
 
+// Resident CTAs per SM the register budget is sized for.
+constexpr int min_blocks(int mt) {
+    return kConsumerWarps <= 8 ? (mt == 1 ? 3 : 2) : (kConsumerWarps <= 12 ? 2 : 1);
+}
+
 template <int FMT, int MT, int MAXI>
-__global__ void __launch_bounds__(kThreads, kConsumerWarps > 8 ? 1 : (MT == 1 ? 3 : 2))
+__global__ void __launch_bounds__(kThreads, min_blocks(MT))
 gemv_kernel(const Batch<MAXI> p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
     uint64_t* empty = full + p.stages;
     uint8_t* xbuf = smem + p.x_off;
-    float* xsum = reinterpret_cast<float*>(smem + p.xsum_off);
+    float4* xmeta = reinterpret_cast<float4*>(smem + p.xmeta_off);
     const long long lo = (long long)blockIdx.x * p.total / gridDim.x;
     const long long hi = (long long)(blockIdx.x + 1) * p.total / gridDim.x;
 
@@ -393,7 +424,7 @@ gemv_kernel(const Batch<MAXI> p) {
         if (ra >= rb) continue;
         if (!first) asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
         first = false;
-        stage_x<FMT, MT>(it, p.m0, p.mrows, xbuf, xsum, tid);
+        stage_x<FMT, MT>(it, p.m0, p.mrows, xbuf, xmeta, tid);
         asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
         RQ_PHASE_MARK(2);
         const int T = it.T, RW = it.RW, KS = it.KS;
@@ -410,13 +441,13 @@ gemv_kernel(const Batch<MAXI> p) {
             if (wfirst < rg) {                           // warp-uniform
                 const uint32_t st_s = smem_s + (uint32_t)s * p.stage_bytes;
                 if (RW == 4)
-                    gemv_group<FMT, MT, 4>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows,
+                    gemv_group<FMT, MT, 4>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xmeta_off, p.m0, p.mrows,
                                            lane, rbase, slice, red);
                 else if (RW == 2)
-                    gemv_group<FMT, MT, 2>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows,
+                    gemv_group<FMT, MT, 2>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xmeta_off, p.m0, p.mrows,
                                            lane, rbase, slice, red);
                 else
-                    gemv_group<FMT, MT, 1>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xsum_off, p.m0, p.mrows,
+                    gemv_group<FMT, MT, 1>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xmeta_off, p.m0, p.mrows,
                                            lane, rbase, slice, red);
             }
             __syncwarp();
@@ -444,7 +475,10 @@ gemv_kernel(const Batch<MAXI> p) {
 #define RQ_GEMV_BATCH_CTAS_PER_SM 2
 #endif
 constexpr size_t kSmemTarget = 72 * 1024;
-constexpr size_t kSmemBatch = 100 * 1024;
+#ifndef RQ_GEMV_SMEM_BATCH_KB
+#define RQ_GEMV_SMEM_BATCH_KB 100
+#endif
+constexpr size_t kSmemBatch = RQ_GEMV_SMEM_BATCH_KB * 1024;
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemAttr = kSmemLimit + 1024;
 
@@ -487,7 +521,8 @@ Layout layout_of(int K) {
     while (l.T > 1 && (hcpr % l.T) != 0) l.T >>= 1;
     const int hj_all = hcpr / l.T;
     l.KS = 1;
-    while (l.T == 32 && l.KS * 2 <= kConsumerWarps && hj_all % (l.KS * 2) == 0 && hj_all / (l.KS * 2) >= 2) l.KS *= 2;
+    while (l.T == 32 && kConsumerWarps % (l.KS * 2) == 0 && hj_all % (l.KS * 2) == 0 && hj_all / (l.KS * 2) >= 2)
+        l.KS *= 2;
     l.HJ = hj_all / l.KS;
     l.teams = (kConsumerWarps / l.KS) * (32 / l.T);
     return l;
@@ -512,8 +547,8 @@ bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b,
     int rho = 1;
     while (((size_t)rho * srb) % 16 != 0) rho <<= 1;     // srb is even, so rho <= 8
     auto stage_bytes = [&](int R) { return round16((size_t)R * crb) + round16((size_t)R * srb); };
-    x_b = (size_t)MT * K * (w4 ? 2 : 4) + (size_t)MT * hcpr * 4;
-    int Rg = l.teams * RW;                               // a power of two
+    x_b = (size_t)MT * K * (w4 ? 2 : 4) + (w4 ? (size_t)MT * hcpr * 16 : 0);
+    int Rg = l.teams * RW;
     while (Rg > rho && Rg > RW && x_b + 2 * stage_bytes(Rg) + 64 > kSmemLimit) Rg >>= 1;
     if (Rg % rho != 0 || x_b + stage_bytes(Rg) + 64 > kSmemLimit) return false;
     it.K = K;
@@ -553,9 +588,12 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
         it.cost1 = total;
         units_min = units_min < 0 || U < units_min ? U : units_min;
         sb = s1 > sb ? s1 : sb;
-        const size_t q = (size_t)MT * a[i].K * (FMT != kFmtW8G16 ? 2 : 4), s = (size_t)MT * (a[i].K / 32) * 4;
+        const size_t q = (size_t)MT * a[i].K * (FMT != kFmtW8G16 ? 2 : 4);
         xq = q > xq ? q : xq;
-        xs = s > xs ? s : xs;
+        if constexpr (FMT != kFmtW8G16) {                // x metadata, int4 formats
+            const size_t s = (size_t)MT * (a[i].K / 32) * 16;
+            xs = s > xs ? s : xs;
+        }
         const size_t rd = it.KS > 1 ? round16((size_t)it.Rg * MT * it.KS * 4) : 0;
         red = rd > red ? rd : red;
     }
@@ -577,8 +615,8 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
     p.stages = stages;
     p.stage_bytes = (uint32_t)sb;
     p.x_off = (uint32_t)(stages * sb);
-    p.xsum_off = (uint32_t)(p.x_off + xq);
-    p.red_off = (uint32_t)round16(p.xsum_off + xs);
+    p.xmeta_off = (uint32_t)(p.x_off + xq);
+    p.red_off = (uint32_t)round16(p.xmeta_off + xs);
     p.red_bytes = (uint32_t)red;
     p.bar_off = (uint32_t)round16(p.red_off + 2 * red);
     const size_t smem = p.bar_off + 2 * stages * sizeof(uint64_t);

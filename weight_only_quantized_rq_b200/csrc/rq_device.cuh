@@ -138,6 +138,11 @@ __device__ __forceinline__ float4 lds128f_a(uint32_t a) {
     asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
     return v;
 }
+__device__ __forceinline__ float2 lds64f_a(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
 __device__ __forceinline__ uint32_t lds32_a(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -311,20 +316,20 @@ __device__ __forceinline__ float fma_f16(uint32_t a, uint32_t b, float c) {
 }
 
 // One code word against x_0..x_7 (fp16, natural-order pairs X.x = (x0, x1),
-// X.y = (x2, x3), X.z = (x4, x5), X.w = (x6, x7)): even k go to lo0/lo1 as
-// (1024 + u_k) x_k, odd k to hi0/hi1 as (1024 + 16 u_k) x_k.
-__device__ __forceinline__ void dot8_w4_f16(uint32_t w, uint4 X, float& lo0, float& lo1, float& hi0, float& hi1) {
+// X.y = (x2, x3), X.z = (x4, x5), X.w = (x6, x7)): lo += (1024 + u_k) x_k over
+// even k, hi += (1024 + 16 u_k) x_k over odd k.
+__device__ __forceinline__ void dot8_w4_f16(uint32_t w, uint4 X, float& lo, float& hi) {
     const uint32_t v = w >> 8;
     const uint32_t p0 = lop_or_mask(w, 0x000F000Fu), p1 = lop_or_mask(w, 0x00F000F0u);
     const uint32_t p2 = lop_or_mask(v, 0x000F000Fu), p3 = lop_or_mask(v, 0x00F000F0u);
-    lo0 = fma_f16<0, 0>(p0, X.x, lo0);   // k0
-    lo1 = fma_f16<1, 0>(p0, X.z, lo1);   // k4
-    hi0 = fma_f16<0, 1>(p1, X.x, hi0);   // k1
-    hi1 = fma_f16<1, 1>(p1, X.z, hi1);   // k5
-    lo0 = fma_f16<0, 0>(p2, X.y, lo0);   // k2
-    lo1 = fma_f16<1, 0>(p2, X.w, lo1);   // k6
-    hi0 = fma_f16<0, 1>(p3, X.y, hi0);   // k3
-    hi1 = fma_f16<1, 1>(p3, X.w, hi1);   // k7
+    lo = fma_f16<0, 0>(p0, X.x, lo);   // k0
+    hi = fma_f16<0, 1>(p1, X.x, hi);   // k1
+    lo = fma_f16<0, 0>(p2, X.y, lo);   // k2
+    hi = fma_f16<0, 1>(p3, X.y, hi);   // k3
+    lo = fma_f16<1, 0>(p0, X.z, lo);   // k4
+    hi = fma_f16<1, 1>(p1, X.z, hi);   // k5
+    lo = fma_f16<1, 0>(p2, X.w, lo);   // k6
+    hi = fma_f16<1, 1>(p3, X.w, hi);   // k7
 }
 
 // int8 codes. Byte k of a word is the code u = q + 128 of weight k. Each byte

@@ -91,41 +91,86 @@ __device__ __forceinline__ void item_units(const Item& it, long long lo, long lo
     ub = (int)first_at_or_after(hi);
 }
 
+// Bytes of the x metadata of the int4 formats for K and MT activation rows:
+// per row m and half-chunk h a float2 {z, sx}, then the per-row factors f[m],
+// then a word per consumer warp and row for the max reduction.
+__host__ __device__ constexpr size_t xmeta_bytes(int K, int MT) {
+    return (size_t)MT * (K / 32) * 8 + 16 + (size_t)kConsumerWarps * MT * 4;
+}
+
 // Staged x for one product and activation rows [m0, m0 + MT).
-//  int4 formats: fp16 quads in natural order (quad q = x[8q .. 8q+7]), each
-//  half-chunk h (32 values) scaled by its own power of two 2^e_h so that its
-//  largest |x| lies in [2^14, 2^15) (exact for every value that stays a
-//  normal fp16, i.e. all but those 2^28 times smaller than the largest), and
-//  a float4 per half-chunk {z, sx, f, 0}: f = 2^-e_h, sx = sum of the scaled
-//  values, z = the code offsets' share (g64: 1032 * sum over even k + 72 *
-//  sum over odd k; sb32: 1024 / 64), summed from the fp16 values the products
-//  use.
+//  int4 formats: fp16 quads in natural order (quad q = x[8q .. 8q+7]); row m
+//  scaled by the power of two 2^e_m that puts its largest |x| in [2^14, 2^15)
+//  (exact for every value no more than 2^32 times smaller than the largest),
+//  with f[m] = 2^-e_m and per half-chunk h: sx = the sum of the scaled values,
+//  z = the code offsets' share (g64: 1032 * sum over even k + 72 * sum over
+//  odd k; sb32: 1024 / 64), both summed from the fp16 values the products use.
 //  int8 format: fp32 quads (quad q = x[4q .. 4q+3]).
+// Called by all consumer threads; contains consumer barriers.
 template <int FMT, int MT>
-__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xbuf, float4* xmeta, int tid) {
+__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xbuf, uint8_t* xmeta, int tid) {
     constexpr bool kW4 = FMT != kFmtW8G16;
+    constexpr int kT = kConsumerWarps * 32;
     const int hcpr = it.K >> 5;
-    for (int i = tid; i < MT * hcpr; i += kConsumerWarps * 32) {
-        const int m = i / hcpr, h = i - m * hcpr;
-        uint4 v[4] = {};
+    auto load = [&](int m, int h, uint4 (&v)[4]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = make_uint4(0u, 0u, 0u, 0u);
         if (m < mrows) {
             const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)h * 32);
 #pragma unroll
             for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
         }
-        uint32_t* w = reinterpret_cast<uint32_t*>(v);
-        if (kW4) {
-            uint32_t mb = 0;
+    };
+    if constexpr (kW4) {
+        float2* zx = reinterpret_cast<float2*>(xmeta);
+        float* fm = reinterpret_cast<float*>(xmeta + (size_t)MT * hcpr * 8);
+        uint32_t* wmax = reinterpret_cast<uint32_t*>(xmeta + (size_t)MT * hcpr * 8 + 16);
+        // largest |x| bit pattern of each row (bf16 magnitudes order as integers)
+        uint32_t mb[MT];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
-            int e = 0;
-            if (mb != 0) e = min(126, max(-126, 14 - ((int)(mb >> 7) - 127)));
-            const float up = __int_as_float((e + 127) << 23);
+        for (int m = 0; m < MT; ++m) mb[m] = 0u;
+        for (int i = tid; i < MT * hcpr; i += kT) {
+            const int m = i / hcpr, h = i - m * hcpr;
+            uint4 v[4];
+            load(m, h, v);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
+            uint32_t t = 0u;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t = max(t, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
+#pragma unroll
+            for (int mm = 0; mm < MT; ++mm)
+                if (mm == m) mb[mm] = max(mb[mm], t);
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const uint32_t r = __reduce_max_sync(0xffffffffu, mb[m]);
+            if ((tid & 31) == 0) wmax[(tid >> 5) * MT + m] = r;
+        }
+        asm volatile("bar.sync 1, %0;" :: "n"(kT) : "memory");
+        float up[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            uint32_t r = 0u;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) r = max(r, wmax[w * MT + m]);
+            const int e = r != 0u ? min(126, max(-126, 14 - ((int)(r >> 7) - 127))) : 0;
+            up[m] = __int_as_float((e + 127) << 23);
+            if (tid == 0) fm[m] = __int_as_float((127 - e) << 23);
+        }
+        for (int i = tid; i < MT * hcpr; i += kT) {
+            const int m = i / hcpr, h = i - m * hcpr;
+            uint4 v[4];
+            load(m, h, v);
+            uint32_t* w = reinterpret_cast<uint32_t*>(v);
+            float u = up[0];
+#pragma unroll
+            for (int mm = 1; mm < MT; ++mm)
+                if (mm == m) u = up[mm];
             float se = 0.0f, so = 0.0f;                  // even-k and odd-k sums
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
-                const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+                const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), u));
+                const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), u));
                 se = __fadd_rn(se, __half2float(a));
                 so = __fadd_rn(so, __half2float(b));
                 w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
@@ -135,8 +180,14 @@ __device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8
             for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[q];
             const float z = FMT == kFmtW4G64 ? __fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so))
                                              : __fmaf_rn(1024.0f, se, __fmul_rn(64.0f, so));
-            xmeta[(size_t)m * hcpr + h] = make_float4(z, __fadd_rn(se, so), __int_as_float((127 - e) << 23), 0.0f);
-        } else {
+            zx[(size_t)m * hcpr + h] = make_float2(z, __fadd_rn(se, so));
+        }
+    } else {
+        for (int i = tid; i < MT * hcpr; i += kT) {
+            const int m = i / hcpr, h = i - m * hcpr;
+            uint4 v[4];
+            load(m, h, v);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
             float4* dst = reinterpret_cast<float4*>(xbuf) + (size_t)m * 8 * hcpr + h;
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -169,7 +220,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
     // x quads: (m * Q + q) * hcpr + h, Q = 4 (bf16) or 8 (fp32) quads per half-chunk
     const uint32_t xstride = (uint32_t)hcpr * 16u;
     const uint32_t xa0 = x_s + (uint32_t)li * 16u;
-    const uint32_t xm0 = xmeta_s + (uint32_t)li * 16u;
+    const uint32_t xm0 = xmeta_s + (uint32_t)li * 8u;
     float yacc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
@@ -197,9 +248,9 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             for (int u = 0; u < U; ++u) {
                 if (u > 0 && hj + u >= HJ) break;
                 const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
-                float4 xm[MT];
+                float2 xm[MT];                           // {z, sx}
 #pragma unroll
-                for (int m = 0; m < MT; ++m) xm[m] = lds128f_a(xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * 16u);
+                for (int m = 0; m < MT; ++m) xm[m] = lds64f_a(xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * 8u);
                 uint4 c[RW];
                 float sA[RW], sB[RW];
 #pragma unroll
@@ -218,40 +269,44 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                         sB[r] = __fmul_rn(dm, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
                     }
                 }
-                // two accumulators for even k ((1024 + u) x) and two for odd k
-                // ((1024 + 16 u) x) per row and m, whatever the launch shape, so
-                // a row's sums (and results) do not depend on RW or on batching
-                float lo0[RW][MT], lo1[RW][MT], hi0[RW][MT], hi1[RW][MT];
+                // one accumulator for even k ((1024 + u) x), started at -z, and
+                // one for odd k ((1024 + 16 u) x) per row and m, whatever the
+                // launch shape, so a row's sums do not depend on RW or batching
+                float lo[RW][MT], hi[RW][MT];
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) lo0[r][m] = lo1[r][m] = hi0[r][m] = hi1[r][m] = 0.0f;
+                    for (int m = 0; m < MT; ++m) {
+                        lo[r][m] = -xm[m].x;
+                        hi[r][m] = 0.0f;
+                    }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         const uint4 X = lds128_a(xa0 + dh * 16u + (uint32_t)(m * 4 + i) * xstride);
 #pragma unroll
-                        for (int r = 0; r < RW; ++r)
-                            dot8_w4_f16(word_of(c[r], i), X, lo0[r][m], lo1[r][m], hi0[r][m], hi1[r][m]);
+                        for (int r = 0; r < RW; ++r) dot8_w4_f16(word_of(c[r], i), X, lo[r][m], hi[r][m]);
                     }
                 }
-                // sum_k q_k x'_k = lo + hi / 16 - z; scaled back by f = 2^-e_h
+                // sum_k q_k x'_k (g64) or sum_k u_k x'_k (sb32) = lo + hi / 16
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
-                        const float a = __fmaf_rn(__fadd_rn(hi0[r][m], hi1[r][m]), 0.0625f,
-                                                  __fadd_rn(lo0[r][m], lo1[r][m]));
-                        const float t = __fsub_rn(a, xm[m].x);
-                        if (FMT == kFmtW4G64) {
-                            yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].z), t, yacc[r][m]);
-                        } else {
-                            const float v = __fmaf_rn(-sB[r], xm[m].y, __fmul_rn(sA[r], t));
-                            yacc[r][m] = __fmaf_rn(xm[m].z, v, yacc[r][m]);
-                        }
+                        const float a = __fmaf_rn(hi[r][m], 0.0625f, lo[r][m]);
+                        yacc[r][m] = __fmaf_rn(sA[r], a, yacc[r][m]);
+                        if (FMT == kFmtW4SB32) yacc[r][m] = __fmaf_rn(-sB[r], xm[m].y, yacc[r][m]);
                     }
             }
+        }
+        // back from the scaled x domain: y = f[m] * sum
+        const uint32_t f_s = xmeta_s + (uint32_t)(MT * hcpr * 8);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const float f = ldsf_a(f_s + (uint32_t)m * 4u);
+#pragma unroll
+            for (int r = 0; r < RW; ++r) yacc[r][m] = __fmul_rn(yacc[r][m], f);
         }
     } else {
         // int8 group 16: 32 code bytes per row and half-chunk = groups 2h, 2h+1;
@@ -361,7 +416,7 @@ gemv_kernel(const Batch<MAXI> p) {
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
     uint64_t* empty = full + p.stages;
     uint8_t* xbuf = smem + p.x_off;
-    float4* xmeta = reinterpret_cast<float4*>(smem + p.xmeta_off);
+    uint8_t* xmeta = smem + p.xmeta_off;
     const long long lo = (long long)blockIdx.x * p.total / gridDim.x;
     const long long hi = (long long)(blockIdx.x + 1) * p.total / gridDim.x;
 
@@ -541,13 +596,12 @@ int rw_allowed(int fmt, int K) {
 // not fit.
 bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b, size_t& x_b) {
     const bool w4 = fmt != kFmtW8G16;
-    const int hcpr = K / 32;
     const Layout l = layout_of(K);
     const size_t crb = code_row_bytes(fmt, K), srb = scale_row_bytes(fmt, K);
     int rho = 1;
     while (((size_t)rho * srb) % 16 != 0) rho <<= 1;     // srb is even, so rho <= 8
     auto stage_bytes = [&](int R) { return round16((size_t)R * crb) + round16((size_t)R * srb); };
-    x_b = (size_t)MT * K * (w4 ? 2 : 4) + (w4 ? (size_t)MT * hcpr * 16 : 0);
+    x_b = (size_t)MT * K * (w4 ? 2 : 4) + (w4 ? round16(xmeta_bytes(K, MT)) : 0);
     int Rg = l.teams * RW;
     while (Rg > rho && Rg > RW && x_b + 2 * stage_bytes(Rg) + 64 > kSmemLimit) Rg >>= 1;
     if (Rg % rho != 0 || x_b + stage_bytes(Rg) + 64 > kSmemLimit) return false;
@@ -591,7 +645,7 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
         const size_t q = (size_t)MT * a[i].K * (FMT != kFmtW8G16 ? 2 : 4);
         xq = q > xq ? q : xq;
         if constexpr (FMT != kFmtW8G16) {                // x metadata, int4 formats
-            const size_t s = (size_t)MT * (a[i].K / 32) * 16;
+            const size_t s = round16(xmeta_bytes(a[i].K, MT));
             xs = s > xs ? s : xs;
         }
         const size_t rd = it.KS > 1 ? round16((size_t)it.Rg * MT * it.KS * 4) : 0;

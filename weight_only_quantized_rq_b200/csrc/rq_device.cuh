@@ -23,6 +23,7 @@ enum : unsigned {
     kStatusSlotWait = 1u << 1,   // waited too long for a ring slot to free
     kStatusMmaWait = 1u << 2,    // waited too long for a tensor-core commit
     kStatusTmem = 1u << 3,       // TMEM allocation did not succeed
+    kStatusXWait = 1u << 4,      // waited too long for a staged activation buffer
 };
 
 // One word per translation unit (internal linkage, so no device linking is
@@ -70,14 +71,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete may be
+// suspended for up to `hint_ns` (or until the phase completes) instead of the
+// system-dependent default, so waiting warps leave the issue slots to the
+// warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Gives up after
 // kWaitLimitNs, ORs `flag` into the device status word and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned flag) {
+// With nap_ns > 0 the warp sleeps that long between polls: for waits off the
+// critical path (a producer waiting for a free slot), so that polling does
+// not take issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned flag,
+                                                  unsigned nap_ns = 0u) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (nap_ns) __nanosleep(nap_ns);
+        if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+        if ((it & 15u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicOr(&g_status, flag);
             return false;
         }

@@ -51,7 +51,14 @@ namespace {
 #define RQ_GEMV_WARPS 8
 #endif
 constexpr int kConsumerWarps = RQ_GEMV_WARPS;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kProducerWarp = kConsumerWarps;         // issues the weight copies
+constexpr int kStagerWarp = kConsumerWarps + 1;       // stages x
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
+#ifndef RQ_PRODUCER_NAP_NS
+#define RQ_PRODUCER_NAP_NS 256
+#endif
+constexpr unsigned kProducerNapNs = RQ_PRODUCER_NAP_NS;   // poll interval of the producer's slot waits
+constexpr unsigned kStagerNapNs = 512;                   // and of the x stager's buffer waits
 
 struct Item {                  // one product of a launch
     const uint16_t* x;         // bf16 bits [M][K]
@@ -73,8 +80,12 @@ template <int MAXI>
 struct Batch {
     int count, m0, mrows;      // items; activation rows [m0, m0 + mrows) of every item
     int stages;
+    int nxb;                   // staged-x buffers (2, or 1 when two do not fit)
     long long total;           // packed bytes of all items
-    uint32_t stage_bytes, x_off, xmeta_off, red_off, red_bytes, bar_off;
+    uint32_t stage_bytes;      // weight ring: stages * stage_bytes at offset 0
+    uint32_t x_off, x_bytes;   // nxb staged-x buffers (x, then its metadata)
+    uint32_t red_off, red_bytes;  // per stage: k-slice partial sums
+    uint32_t bar_off;          // full[stages], empty[stages], xfull[2], xempty[2]
     Item it[MAXI];
 };
 
@@ -91,108 +102,82 @@ __device__ __forceinline__ void item_units(const Item& it, long long lo, long lo
     ub = (int)first_at_or_after(hi);
 }
 
-// Bytes of the x metadata of the int4 formats for K and MT activation rows:
-// per row m and half-chunk h a float2 {z, sx}, then the per-row factors f[m],
-// then a word per consumer warp and row for the max reduction.
-__host__ __device__ constexpr size_t xmeta_bytes(int K, int MT) {
-    return (size_t)MT * (K / 32) * 8 + 16 + (size_t)kConsumerWarps * MT * 4;
+// Bytes of one staged-x buffer for K and MT activation rows: the values
+// (fp16 for the int4 formats, fp32 for int8), then for the int4 formats a
+// metadata record per row m and half-chunk h (g64: float2, sb32: float4).
+__host__ __device__ constexpr size_t xvals_bytes(int fmt, int K, int MT) {
+    return (size_t)MT * K * (fmt != kFmtW8G16 ? 2 : 4);
+}
+__host__ __device__ constexpr size_t xbuf_bytes(int fmt, int K, int MT) {
+    return xvals_bytes(fmt, K, MT) + (size_t)MT * (K / 32) * (fmt == kFmtW4G64 ? 8 : fmt == kFmtW4SB32 ? 16 : 0);
 }
 
-// Staged x for one product and activation rows [m0, m0 + MT).
-//  int4 formats: fp16 quads in natural order (quad q = x[8q .. 8q+7]); row m
-//  scaled by the power of two 2^e_m that puts its largest |x| in [2^14, 2^15)
-//  (exact for every value no more than 2^32 times smaller than the largest),
-//  with f[m] = 2^-e_m and per half-chunk h: sx = the sum of the scaled values,
+// Stages x for one product and activation rows [m0, m0 + MT); run by one
+// warp, lane i taking half-chunks i, i + 32, ...
+//  int4 formats: fp16 quads in natural order (quad q = x[8q .. 8q+7]), each
+//  half-chunk h (32 values) scaled by the power of two 2^e_h that puts its
+//  largest |x| in [2^14, 2^15) (exact for every value no more than 2^32 times
+//  smaller than the largest), and per half-chunk f = 2^-e_h and
 //  z = the code offsets' share (g64: 1032 * sum over even k + 72 * sum over
-//  odd k; sb32: 1024 / 64), both summed from the fp16 values the products use.
+//  odd k; sb32: 1024 / 64), summed from the fp16 values the products use;
+//  g64 keeps {z, f}, sb32 {z, f * sum, f, 0}.
 //  int8 format: fp32 quads (quad q = x[4q .. 4q+3]).
-// Called by all consumer threads; contains consumer barriers.
 template <int FMT, int MT>
-__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xbuf, uint8_t* xmeta, int tid) {
+__device__ __forceinline__ void stage_x_warp(const Item& it, int m0, int mrows, uint8_t* xb, int lane) {
     constexpr bool kW4 = FMT != kFmtW8G16;
-    constexpr int kT = kConsumerWarps * 32;
-    const int hcpr = it.K >> 5;
-    auto load = [&](int m, int h, uint4 (&v)[4]) {
+    const int hcpr = it.K >> 5, n = MT * hcpr;
+    uint8_t* meta = xb + xvals_bytes(FMT, it.K, MT);
+    for (int i0 = lane; i0 < n; i0 += 64) {
+        uint4 v[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (m < mrows) {
-            const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)h * 32);
+        for (int u = 0; u < 2; ++u) {               // both loads in flight before use
+            const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
-        }
-    };
-    if constexpr (kW4) {
-        float2* zx = reinterpret_cast<float2*>(xmeta);
-        float* fm = reinterpret_cast<float*>(xmeta + (size_t)MT * hcpr * 8);
-        uint32_t* wmax = reinterpret_cast<uint32_t*>(xmeta + (size_t)MT * hcpr * 8 + 16);
-        // largest |x| bit pattern of each row (bf16 magnitudes order as integers)
-        uint32_t mb[MT];
+            for (int j = 0; j < 4; ++j) v[u][j] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < n && m < mrows) {
+                const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)h * 32);
 #pragma unroll
-        for (int m = 0; m < MT; ++m) mb[m] = 0u;
-        for (int i = tid; i < MT * hcpr; i += kT) {
-            const int m = i / hcpr, h = i - m * hcpr;
-            uint4 v[4];
-            load(m, h, v);
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
-            uint32_t t = 0u;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) t = max(t, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
-#pragma unroll
-            for (int mm = 0; mm < MT; ++mm)
-                if (mm == m) mb[mm] = max(mb[mm], t);
-        }
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const uint32_t r = __reduce_max_sync(0xffffffffu, mb[m]);
-            if ((tid & 31) == 0) wmax[(tid >> 5) * MT + m] = r;
-        }
-        asm volatile("bar.sync 1, %0;" :: "n"(kT) : "memory");
-        float up[MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            uint32_t r = 0u;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) r = max(r, wmax[w * MT + m]);
-            const int e = r != 0u ? min(126, max(-126, 14 - ((int)(r >> 7) - 127))) : 0;
-            up[m] = __int_as_float((e + 127) << 23);
-            if (tid == 0) fm[m] = __int_as_float((127 - e) << 23);
-        }
-        for (int i = tid; i < MT * hcpr; i += kT) {
-            const int m = i / hcpr, h = i - m * hcpr;
-            uint4 v[4];
-            load(m, h, v);
-            uint32_t* w = reinterpret_cast<uint32_t*>(v);
-            float u = up[0];
-#pragma unroll
-            for (int mm = 1; mm < MT; ++mm)
-                if (mm == m) u = up[mm];
-            float se = 0.0f, so = 0.0f;                  // even-k and odd-k sums
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), u));
-                const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), u));
-                se = __fadd_rn(se, __half2float(a));
-                so = __fadd_rn(so, __half2float(b));
-                w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+                for (int j = 0; j < 4; ++j) v[u][j] = __ldg(src + j);
             }
-            uint4* dst = reinterpret_cast<uint4*>(xbuf) + (size_t)m * 4 * hcpr + h;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[q];
-            const float z = FMT == kFmtW4G64 ? __fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so))
-                                             : __fmaf_rn(1024.0f, se, __fmul_rn(64.0f, so));
-            zx[(size_t)m * hcpr + h] = make_float2(z, __fadd_rn(se, so));
         }
-    } else {
-        for (int i = tid; i < MT * hcpr; i += kT) {
-            const int m = i / hcpr, h = i - m * hcpr;
-            uint4 v[4];
-            load(m, h, v);
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
-            float4* dst = reinterpret_cast<float4*>(xbuf) + (size_t)m * 8 * hcpr + h;
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                dst[(size_t)q * hcpr] = make_float4(bf16lo_f32(w[2 * q]), bf16hi_f32(w[2 * q]),
-                                                    bf16lo_f32(w[2 * q + 1]), bf16hi_f32(w[2 * q + 1]));
+        for (int u = 0; u < 2; ++u) {
+            const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
+            if (i >= n) break;
+            uint32_t* w = reinterpret_cast<uint32_t*>(v[u]);
+            if constexpr (kW4) {
+                uint32_t mb = 0u;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
+                const int e = mb != 0u ? min(126, max(-126, 14 - ((int)(mb >> 7) - 127))) : 0;
+                const float up = __int_as_float((e + 127) << 23), f = __int_as_float((127 - e) << 23);
+                float se = 0.0f, so = 0.0f;              // even-k and odd-k sums
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
+                    const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+                    se = __fadd_rn(se, __half2float(a));
+                    so = __fadd_rn(so, __half2float(b));
+                    w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(xb) + (size_t)m * 4 * hcpr + h;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[u][q];
+                if (FMT == kFmtW4G64) {
+                    const float z = __fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so));
+                    reinterpret_cast<float2*>(meta)[(size_t)m * hcpr + h] = make_float2(z, f);
+                } else {
+                    const float z = __fmaf_rn(1024.0f, se, __fmul_rn(64.0f, so));
+                    reinterpret_cast<float4*>(meta)[(size_t)m * hcpr + h] =
+                        make_float4(z, __fmul_rn(f, __fadd_rn(se, so)), f, 0.0f);
+                }
+            } else {
+                float4* dst = reinterpret_cast<float4*>(xb) + (size_t)m * 8 * hcpr + h;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[(size_t)q * hcpr] = make_float4(bf16lo_f32(w[2 * q]), bf16hi_f32(w[2 * q]),
+                                                        bf16lo_f32(w[2 * q + 1]), bf16hi_f32(w[2 * q + 1]));
+            }
         }
     }
 }
@@ -206,13 +191,12 @@ __device__ __forceinline__ uint32_t word_of(const uint4& c, int i) {
 // Rows past rg (the group's last rows) lie inside the stage buffer, which
 // always has room for Rg rows; they hold stale bytes whose results are never
 // stored.
-template <int FMT, int MT, int RW>
-__device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s,
-                                           uint32_t xmeta_s, int m0, int mrows, int lane, int rbase, int slice,
+template <int FMT, int MT, int RW, int TT>
+__device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s, int m0, int mrows, int lane, int rbase, int slice,
                                            float* red) {
     constexpr bool kW4 = FMT != kFmtW8G16;
     constexpr int U = RW == 1 ? 2 : 1;                   // half-chunks per iteration
-    const int hcpr = it.K >> 5, T = it.T, HJ = it.HJ;
+    const int hcpr = it.K >> 5, T = TT ? TT : it.T, HJ = it.HJ;   // TT: team lanes fixed at compile time
     const int li = lane & (T - 1);
     const int hoff = slice * HJ;                         // this warp's k-slice of the row
     const uint32_t crb = it.crb, srb = it.srb;
@@ -220,7 +204,8 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
     // x quads: (m * Q + q) * hcpr + h, Q = 4 (bf16) or 8 (fp32) quads per half-chunk
     const uint32_t xstride = (uint32_t)hcpr * 16u;
     const uint32_t xa0 = x_s + (uint32_t)li * 16u;
-    const uint32_t xm0 = xmeta_s + (uint32_t)li * 8u;
+    constexpr uint32_t kMeta = FMT == kFmtW4G64 ? 8u : 16u;          // metadata record bytes
+    const uint32_t xm0 = x_s + (uint32_t)xvals_bytes(FMT, it.K, MT) + (uint32_t)li * kMeta;
     float yacc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
@@ -248,9 +233,17 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             for (int u = 0; u < U; ++u) {
                 if (u > 0 && hj + u >= HJ) break;
                 const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
-                float2 xm[MT];                           // {z, sx}
+                float4 xm[MT];                           // g64: {z, f}; sb32: {z, f * sum, f}
 #pragma unroll
-                for (int m = 0; m < MT; ++m) xm[m] = lds64f_a(xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * 8u);
+                for (int m = 0; m < MT; ++m) {
+                    const uint32_t a = xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * kMeta;
+                    if (FMT == kFmtW4G64) {
+                        const float2 t = lds64f_a(a);
+                        xm[m] = make_float4(t.x, t.y, 0.0f, 0.0f);
+                    } else {
+                        xm[m] = lds128f_a(a);
+                    }
+                }
                 uint4 c[RW];
                 float sA[RW], sB[RW];
 #pragma unroll
@@ -289,24 +282,21 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                         for (int r = 0; r < RW; ++r) dot8_w4_f16(word_of(c[r], i), X, lo[r][m], hi[r][m]);
                     }
                 }
-                // sum_k q_k x'_k (g64) or sum_k u_k x'_k (sb32) = lo + hi / 16
+                // sum_k q_k x'_k (g64) or sum_k u_k x'_k (sb32) = lo + hi / 16;
+                // back to x's scale with f = 2^-e_h
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         const float a = __fmaf_rn(hi[r][m], 0.0625f, lo[r][m]);
-                        yacc[r][m] = __fmaf_rn(sA[r], a, yacc[r][m]);
-                        if (FMT == kFmtW4SB32) yacc[r][m] = __fmaf_rn(-sB[r], xm[m].y, yacc[r][m]);
+                        if (FMT == kFmtW4G64) {
+                            yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].y), a, yacc[r][m]);
+                        } else {
+                            yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].z), a, yacc[r][m]);
+                            yacc[r][m] = __fmaf_rn(-sB[r], xm[m].y, yacc[r][m]);
+                        }
                     }
             }
-        }
-        // back from the scaled x domain: y = f[m] * sum
-        const uint32_t f_s = xmeta_s + (uint32_t)(MT * hcpr * 8);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const float f = ldsf_a(f_s + (uint32_t)m * 4u);
-#pragma unroll
-            for (int r = 0; r < RW; ++r) yacc[r][m] = __fmul_rn(yacc[r][m], f);
         }
     } else {
         // int8 group 16: 32 code bytes per row and half-chunk = groups 2h, 2h+1;
@@ -379,34 +369,89 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                 else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = v;
             }
         }
-        return;
-    }
+    } else {                                             // shuffle tree per row, lane 0 of each team stores
 #pragma unroll
-    for (int r = 0; r < RW; ++r)
+        for (int r = 0; r < RW; ++r)
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            float v = yacc[r][m];
-            for (int o = T >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            yacc[r][m] = v;
-        }
-    if (li == 0) {
+            for (int m = 0; m < MT; ++m) {
+                float v = yacc[r][m];
+                for (int o = T >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                yacc[r][m] = v;
+            }
+        if (li == 0) {
 #pragma unroll
-        for (int r = 0; r < RW; ++r) {
-            const int rr = rbase + r;
-            if (rr < rg)
+            for (int r = 0; r < RW; ++r) {
+                const int rr = rbase + r;
+                if (rr < rg)
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = yacc[r][m];
-                    else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = yacc[r][m];
-                }
+                    for (int m = 0; m < MT; ++m) {
+                        if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = yacc[r][m];
+                        else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = yacc[r][m];
+                    }
+            }
         }
     }
 }
 
-// Resident CTAs per SM the register budget is sized for.
-constexpr int min_blocks(int mt) {
-    return kConsumerWarps <= 8 ? (mt == 1 ? 3 : 2) : (kConsumerWarps <= 12 ? 2 : 1);
+// Consumer view of the weight ring (one copy per warp, in registers).
+struct Ring {
+    uint64_t* full;
+    uint64_t* empty;
+    uint8_t* red;              // per-stage k-slice partial sums
+    uint32_t base;             // shared address of stage 0
+    uint32_t stage_bytes, red_bytes;
+    int stages;
+    int s;                     // stage of the next group
+    uint32_t ph;               // its phase parity
+};
+
+// All groups of rows [ra, rb) of item `it` for this warp: waits for each
+// stage, computes its team's rows, stores the outputs (with KS > 1: the
+// team's slice-0 warp adds the k-slices after a team barrier) and releases
+// the stage. The launch shape (RW, TT) is fixed per item, so the per-item
+// setup stays outside the group loop. False if a bounded wait gave up.
+template <int FMT, int MT, int RW, int TT>
+__device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& ring, uint32_t x_s, int m0,
+                                          int mrows, int warp, int lane) {
+    const int T = TT ? TT : it.T, KS = it.KS, Rg = it.Rg;
+    const int slice = warp % KS;                         // k-slice of this warp (KS > 1 only when T == 32)
+    const int team = warp / KS;                          // warps team*KS .. team*KS+KS-1 share rows
+    const int wteam = team * (32 / T);                   // first lane team of this warp
+    const int rbase = (wteam + lane / T) * RW;           // first row of this lane team in a group
+    const int wfirst = wteam * RW;                       // first row of this warp in a group
+    for (int g0 = ra; g0 < rb; g0 += Rg) {
+        const int s = ring.s;
+        if (!mbar_wait_bounded(&ring.full[s], ring.ph, kStatusTmaWait)) return false;
+        if (++ring.s == ring.stages) {                   // next stage and its phase parity
+            ring.s = 0;
+            ring.ph ^= 1u;
+        }
+        const int rg = min(Rg, rb - g0);
+        if (wfirst < rg) {                               // warp-uniform
+            float* red = reinterpret_cast<float*>(ring.red + (size_t)s * ring.red_bytes);
+            gemv_group<FMT, MT, RW, TT>(it, ring.base + (uint32_t)s * ring.stage_bytes, g0, rg, x_s, m0, mrows,
+                                        lane, rbase, slice, red);
+            if (KS > 1) {
+                asm volatile("bar.sync %0, %1;" :: "r"(1 + team), "r"(KS * 32) : "memory");
+                if (slice == 0 && lane < RW * MT) {
+                    const int r = lane / MT, m = lane - r * MT, rr = wfirst + r;
+                    if (rr < rg && m < mrows) {
+                        const float* q = red + ((size_t)rr * MT + m) * KS;
+                        float v = 0.0f;
+                        for (int k = 0; k < KS; ++k) v += q[k];
+                        it.y[(size_t)(m0 + m) * it.N + g0 + rr] = v;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[s]);     // stage consumed
+    }
+    return true;
 }
+
+// Resident CTAs per SM the register budget is sized for.
+constexpr int min_blocks(int) { return kConsumerWarps <= 12 ? 2 : 1; }
 
 template <int FMT, int MT, int MAXI>
 __global__ void __launch_bounds__(kThreads, min_blocks(MT))
@@ -415,8 +460,8 @@ gemv_kernel(const Batch<MAXI> p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
     uint64_t* empty = full + p.stages;
-    uint8_t* xbuf = smem + p.x_off;
-    uint8_t* xmeta = smem + p.xmeta_off;
+    uint64_t* xfull = empty + p.stages;                  // staged x buffer b ready (32 stager lanes)
+    uint64_t* xempty = xfull + 2;                        // staged x buffer b released (consumer warps)
     const long long lo = (long long)blockIdx.x * p.total / gridDim.x;
     const long long hi = (long long)(blockIdx.x + 1) * p.total / gridDim.x;
 
@@ -425,13 +470,17 @@ gemv_kernel(const Batch<MAXI> p) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&xfull[b], 32);
+            mbar_init(&xempty[b], kConsumerWarps);
+        }
         fence_mbar_init();
     }
     __syncthreads();
     grid_dep_launch();
     RQ_PHASE_MARK(0);
 
-    if (warp == kConsumerWarps) {                        // producer warp
+    if (warp == kProducerWarp) {                         // weight copies into the ring
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();
             int gi = 0;
@@ -445,7 +494,8 @@ gemv_kernel(const Batch<MAXI> p) {
                 const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
                 for (int g0 = ra; g0 < rb; g0 += it.Rg, ++gi) {
                     const int s = gi % p.stages;
-                    if (gi >= p.stages && !mbar_wait_bounded(&empty[s], ((gi / p.stages) - 1) & 1, kStatusSlotWait)) {
+                    if (gi >= p.stages &&
+                        !mbar_wait_bounded(&empty[s], ((gi / p.stages) - 1) & 1, kStatusSlotWait, kProducerNapNs)) {
                         ok = false;
                         break;
                     }
@@ -463,60 +513,67 @@ gemv_kernel(const Batch<MAXI> p) {
         return;
     }
 
+    if (warp == kStagerWarp) {                           // x of each item into alternating buffers
+        grid_dep_wait();                                 // x is written by the previous kernel
+        int xi = 0;
+        for (int i = 0; i < p.count; ++i) {
+            const Item& it = p.it[i];
+            if (it.cost0 >= hi) break;
+            if (it.cost1 <= lo) continue;
+            int ua, ub;
+            item_units(it, lo, hi, ua, ub);
+            if (ua * it.rho >= min(ub * it.rho, it.N)) continue;
+            const int b = xi % p.nxb;
+            if (xi >= p.nxb && !mbar_wait_bounded(&xempty[b], ((xi / p.nxb) - 1) & 1, kStatusXWait, kStagerNapNs))
+                break;
+            stage_x_warp<FMT, MT>(it, p.m0, p.mrows, smem + p.x_off + (size_t)b * p.x_bytes, lane);
+            mbar_arrive(&xfull[b]);                      // each lane: its stores are released
+            ++xi;
+        }
+        return;
+    }
+
     // ---- consumers ---------------------------------------------------------
     const uint32_t smem_s = smem_u32(smem);
-    grid_dep_wait();                                     // x is written by the previous kernel
+    grid_dep_wait();                                     // y may be read by the previous kernel
     RQ_PHASE_MARK(1);
-    int gi = 0;
-    bool first = true;
+    Ring ring;
+    ring.full = full;
+    ring.empty = empty;
+    ring.red = smem + p.red_off;
+    ring.base = smem_s;
+    ring.stage_bytes = p.stage_bytes;
+    ring.red_bytes = p.red_bytes;
+    ring.stages = p.stages;
+    ring.s = 0;
+    ring.ph = 0u;
+    int xi = 0;                                          // items done
     for (int i = 0; i < p.count; ++i) {
-        const Item& it = p.it[i];
+        const Item it = p.it[i];                         // this item's fields in registers
         if (it.cost0 >= hi) break;                       // items are in cost order
         if (it.cost1 <= lo) continue;                    // no overlap: skip without dividing
         int ua, ub;
         item_units(it, lo, hi, ua, ub);
         const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
         if (ra >= rb) continue;
-        if (!first) asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
-        first = false;
-        stage_x<FMT, MT>(it, p.m0, p.mrows, xbuf, xmeta, tid);
-        asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
+        const int b = xi % p.nxb;
+        if (!mbar_wait_bounded(&xfull[b], (xi / p.nxb) & 1, kStatusXWait)) return;
         RQ_PHASE_MARK(2);
-        const int T = it.T, RW = it.RW, KS = it.KS;
-        const int slice = warp % KS;                     // k-slice of this warp (KS > 1 only when T == 32)
-        const int wteam = (warp / KS) * (32 / T);         // first team of this warp
-        const int rbase = (wteam + lane / T) * RW;        // first row of this team in a group
-        const int wfirst = wteam * RW;                    // first row of this warp in a group
-        for (int g0 = ra; g0 < rb; g0 += it.Rg, ++gi) {
-            const int s = gi % p.stages;
-            if (!mbar_wait_bounded(&full[s], (gi / p.stages) & 1, kStatusTmaWait)) return;
-            RQ_PHASE_MARK(3);
-            const int rg = min(it.Rg, rb - g0);
-            float* red = reinterpret_cast<float*>(smem + p.red_off + (gi & 1) * p.red_bytes);
-            if (wfirst < rg) {                           // warp-uniform
-                const uint32_t st_s = smem_s + (uint32_t)s * p.stage_bytes;
-                if (RW == 4)
-                    gemv_group<FMT, MT, 4>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xmeta_off, p.m0, p.mrows,
-                                           lane, rbase, slice, red);
-                else if (RW == 2)
-                    gemv_group<FMT, MT, 2>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xmeta_off, p.m0, p.mrows,
-                                           lane, rbase, slice, red);
-                else
-                    gemv_group<FMT, MT, 1>(it, st_s, g0, rg, smem_s + p.x_off, smem_s + p.xmeta_off, p.m0, p.mrows,
-                                           lane, rbase, slice, red);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);       // stage consumed
-            if (KS > 1) {                                // combine the k-slices of each row
-                asm volatile("bar.sync 1, %0;" :: "n"(kConsumerWarps * 32) : "memory");
-                for (int t = tid; t < rg * MT; t += kConsumerWarps * 32) {
-                    const int rr = t / MT, m = t - rr * MT;
-                    float v = 0.0f;
-                    for (int k = 0; k < KS; ++k) v += red[(size_t)t * KS + k];
-                    if (m < p.mrows) it.y[(size_t)(p.m0 + m) * it.N + g0 + rr] = v;
-                }
-            }
+        const uint32_t x_s = smem_s + p.x_off + (uint32_t)b * p.x_bytes;
+        bool ok;
+        if (it.T == 32) {                                // whole-warp teams: the common case
+            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 32>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 32>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                              : gemv_item<FMT, MT, 1, 32>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
+        } else {
+            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 0>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 0>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                              : gemv_item<FMT, MT, 1, 0>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
         }
+        if (!ok) return;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xempty[b]);          // staged x released
+        ++xi;
     }
     RQ_PHASE_MARK(4);
 }
@@ -531,7 +588,7 @@ gemv_kernel(const Batch<MAXI> p) {
 #endif
 constexpr size_t kSmemTarget = 72 * 1024;
 #ifndef RQ_GEMV_SMEM_BATCH_KB
-#define RQ_GEMV_SMEM_BATCH_KB 100
+#define RQ_GEMV_SMEM_BATCH_KB 112
 #endif
 constexpr size_t kSmemBatch = RQ_GEMV_SMEM_BATCH_KB * 1024;
 constexpr size_t kSmemLimit = 220 * 1024;
@@ -585,26 +642,30 @@ Layout layout_of(int K) {
 
 // Rows per team for a product: the largest of 4, 2, 1 whose group of
 // teams * RW rows stays within 48 KB.
+#ifndef RQ_GEMV_RW_MAX
+#define RQ_GEMV_RW_MAX 4
+#endif
 int rw_allowed(int fmt, int K) {
     const Layout l = layout_of(K);
+    if (RQ_GEMV_RW_MAX < 4) return RQ_GEMV_RW_MAX;
     auto sb = [&](size_t R) { return round16(R * code_row_bytes(fmt, K)) + round16(R * scale_row_bytes(fmt, K)); };
     if (sb((size_t)l.teams * 4) <= 48 * 1024) return 4;
     return sb((size_t)l.teams * 2) <= 48 * 1024 ? 2 : 1;
 }
 
 // Per-item launch geometry for rows-per-team RW; false for a shape that does
-// not fit.
-bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b, size_t& x_b) {
-    const bool w4 = fmt != kFmtW8G16;
+// not fit even with one staged-x buffer.
+bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b) {
     const Layout l = layout_of(K);
     const size_t crb = code_row_bytes(fmt, K), srb = scale_row_bytes(fmt, K);
     int rho = 1;
     while (((size_t)rho * srb) % 16 != 0) rho <<= 1;     // srb is even, so rho <= 8
     auto stage_bytes = [&](int R) { return round16((size_t)R * crb) + round16((size_t)R * srb); };
-    x_b = (size_t)MT * K * (w4 ? 2 : 4) + (w4 ? round16(xmeta_bytes(K, MT)) : 0);
+    auto red_bytes = [&](int R) { return l.KS > 1 ? round16((size_t)R * MT * l.KS * 4) : (size_t)0; };
+    const size_t x1 = round16(xbuf_bytes(fmt, K, MT)) + 256;   // one x buffer, counters, barriers
     int Rg = l.teams * RW;
-    while (Rg > rho && Rg > RW && x_b + 2 * stage_bytes(Rg) + 64 > kSmemLimit) Rg >>= 1;
-    if (Rg % rho != 0 || x_b + stage_bytes(Rg) + 64 > kSmemLimit) return false;
+    while (Rg > rho && Rg > RW && x1 + 2 * (stage_bytes(Rg) + red_bytes(Rg)) > kSmemLimit) Rg >>= 1;
+    if (Rg % rho != 0 || x1 + stage_bytes(Rg) + red_bytes(Rg) > kSmemLimit) return false;
     it.K = K;
     it.N = N;
     it.T = l.T;
@@ -620,70 +681,93 @@ bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b,
     return true;
 }
 
+// Shared-memory plan of a launch: ring of `stages` stages, nxb staged-x
+// buffers, per-stage k-slice partials, barriers. Prefers two
+// x buffers and a size that lets two CTAs share an SM (`want`).
+struct SmemPlan { int stages, nxb; size_t smem; };
+bool plan_smem(size_t sb, size_t xbb, size_t red, size_t want, int max_stages, SmemPlan& o) {
+    auto fixed = [&](int nxb, int st) { return (size_t)nxb * xbb + (size_t)(2 * st + 4) * 8; };
+    auto fits = [&](int nxb, int st, size_t cap) { return st * (sb + red) + fixed(nxb, st) <= cap; };
+    for (size_t cap : {want, kSmemLimit})
+        for (int nxb = 2; nxb >= 1; --nxb) {
+            if (!fits(nxb, cap == want ? 2 : 1, cap)) continue;
+            int st = 1;
+            while (st < max_stages && fits(nxb, st + 1, cap)) ++st;
+            o.stages = st;
+            o.nxb = nxb;
+            o.smem = st * (sb + red) + fixed(nxb, st);
+            return true;
+        }
+    return false;
+}
+
 template <int FMT, int MAXI>
 cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
     const int M = a[0].M;
-    const int MT = M >= 2 ? 2 : 1;
-    Batch<MAXI> p = {};
-    p.count = count;
-    size_t sb = 0, xq = 0, xs = 0, red = 0;
-    long long total = 0, units_min = -1;
-    for (int i = 0; i < count; ++i) {
-        Item& it = p.it[i];
-        size_t s1, x1;
-        if (!plan_item(FMT, a[i].K, a[i].N, MT, rw_allowed(FMT, a[i].K), it, s1, x1)) return cudaErrorInvalidValue;
-        it.x = static_cast<const uint16_t*>(a[i].x);
-        it.codes = static_cast<const uint8_t*>(a[i].codes);
-        it.scales = static_cast<const uint8_t*>(a[i].scales);
-        it.y = a[i].y;
-        it.cost0 = total;
-        const long long U = (it.N + it.rho - 1) / it.rho;
-        total += U * it.ucost;
-        it.cost1 = total;
-        units_min = units_min < 0 || U < units_min ? U : units_min;
-        sb = s1 > sb ? s1 : sb;
-        const size_t q = (size_t)MT * a[i].K * (FMT != kFmtW8G16 ? 2 : 4);
-        xq = q > xq ? q : xq;
-        if constexpr (FMT != kFmtW8G16) {                // x metadata, int4 formats
-            const size_t s = round16(xmeta_bytes(a[i].K, MT));
-            xs = s > xs ? s : xs;
+    for (int MT = M >= 2 ? 2 : 1; MT >= 1; --MT) {
+        Batch<MAXI> p = {};
+        p.count = count;
+        size_t sb = 0, xbb = 0, red = 0;
+        long long total = 0, units_min = -1;
+        bool ok = true;
+        for (int i = 0; i < count && ok; ++i) {
+            Item& it = p.it[i];
+            size_t s1;
+            if (!plan_item(FMT, a[i].K, a[i].N, MT, rw_allowed(FMT, a[i].K), it, s1)) {
+                ok = false;
+                break;
+            }
+            it.x = static_cast<const uint16_t*>(a[i].x);
+            it.codes = static_cast<const uint8_t*>(a[i].codes);
+            it.scales = static_cast<const uint8_t*>(a[i].scales);
+            it.y = a[i].y;
+            it.cost0 = total;
+            const long long U = (it.N + it.rho - 1) / it.rho;
+            total += U * it.ucost;
+            it.cost1 = total;
+            units_min = units_min < 0 || U < units_min ? U : units_min;
+            sb = s1 > sb ? s1 : sb;
+            const size_t xq = round16(xbuf_bytes(FMT, a[i].K, MT));
+            xbb = xq > xbb ? xq : xbb;
+            const size_t rd = it.KS > 1 ? round16((size_t)it.Rg * MT * it.KS * 4) : 0;
+            red = rd > red ? rd : red;
         }
-        const size_t rd = it.KS > 1 ? round16((size_t)it.Rg * MT * it.KS * 4) : 0;
-        red = rd > red ? rd : red;
-    }
-    p.total = total;
-    int grid = sm_count() * (count > 1 ? RQ_GEMV_BATCH_CTAS_PER_SM : RQ_GEMV_SINGLE_CTAS_PER_SM);
-    if (count == 1 && grid > units_min) grid = (int)units_min;
-    const size_t fixed = xq + xs + 2 * red + 64;
-    const size_t want = count > 1 ? kSmemBatch : kSmemTarget;
-    const size_t budget = fixed + 2 * sb <= want ? want : kSmemLimit;
-    int stages = (int)((budget - fixed) / sb);
-    if (stages > 6) stages = 6;
-    if (count == 1) {   // a single product needs no more stages than its largest CTA has groups
-        const Item& it = p.it[0];
-        const long long per = (units_min + grid - 1) / grid * it.rho;
-        const int gmax = (int)((per + it.Rg - 1) / it.Rg);
-        if (stages > gmax) stages = gmax;
-    }
-    if (stages < 1) return cudaErrorInvalidValue;
-    p.stages = stages;
-    p.stage_bytes = (uint32_t)sb;
-    p.x_off = (uint32_t)(stages * sb);
-    p.xmeta_off = (uint32_t)(p.x_off + xq);
-    p.red_off = (uint32_t)round16(p.xmeta_off + xs);
-    p.red_bytes = (uint32_t)red;
-    p.bar_off = (uint32_t)round16(p.red_off + 2 * red);
-    const size_t smem = p.bar_off + 2 * stages * sizeof(uint64_t);
-    if (smem > kSmemAttr) return cudaErrorInvalidValue;
+        SmemPlan sp;
+        if (!ok || !plan_smem(sb, xbb, red, count > 1 ? kSmemBatch : kSmemTarget, 6, sp)) {
+            if (MT == 2) continue;                       // retry one activation row per launch
+            return cudaErrorInvalidValue;
+        }
+        p.total = total;
+        int grid = sm_count() * (count > 1 ? RQ_GEMV_BATCH_CTAS_PER_SM : RQ_GEMV_SINGLE_CTAS_PER_SM);
+        if (count == 1 && grid > units_min) grid = (int)units_min;
+        int stages = sp.stages;
+        if (count == 1) {   // a single product needs no more stages than its largest CTA has groups
+            const Item& it = p.it[0];
+            const long long per = (units_min + grid - 1) / grid * it.rho;
+            const int gmax = (int)((per + it.Rg - 1) / it.Rg);
+            if (stages > gmax) stages = gmax;
+        }
+        p.stages = stages;
+        p.nxb = sp.nxb;
+        p.stage_bytes = (uint32_t)sb;
+        p.x_off = (uint32_t)(stages * sb);
+        p.x_bytes = (uint32_t)xbb;
+        p.red_off = (uint32_t)(p.x_off + sp.nxb * xbb);
+        p.red_bytes = (uint32_t)red;
+        p.bar_off = (uint32_t)(p.red_off + stages * red);
+        const size_t smem = p.bar_off + (size_t)(2 * stages + 4) * sizeof(uint64_t);
+        if (smem > kSmemAttr) return cudaErrorInvalidValue;
 
-    for (int m0 = 0; m0 < M; m0 += MT) {
-        p.m0 = m0;
-        p.mrows = M - m0 < MT ? M - m0 : MT;
-        const cudaError_t e = MT == 2 ? launch_one<FMT, 2, MAXI>(p, smem, grid, st)
-                                      : launch_one<FMT, 1, MAXI>(p, smem, grid, st);
-        if (e != cudaSuccess) return e;
+        for (int m0 = 0; m0 < M; m0 += MT) {
+            p.m0 = m0;
+            p.mrows = M - m0 < MT ? M - m0 : MT;
+            const cudaError_t e = MT == 2 ? launch_one<FMT, 2, MAXI>(p, smem, grid, st)
+                                          : launch_one<FMT, 1, MAXI>(p, smem, grid, st);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
-    return cudaSuccess;
+    return cudaErrorInvalidValue;
 }
 
 template <int FMT>

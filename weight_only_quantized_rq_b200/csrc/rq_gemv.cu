@@ -109,7 +109,7 @@ __host__ __device__ constexpr size_t xvals_bytes(int fmt, int K, int MT) {
     return (size_t)MT * K * (fmt != kFmtW8G16 ? 2 : 4);
 }
 __host__ __device__ constexpr size_t xbuf_bytes(int fmt, int K, int MT) {
-    return xvals_bytes(fmt, K, MT) + (size_t)MT * (K / 32) * (fmt == kFmtW4G64 ? 8 : fmt == kFmtW4SB32 ? 16 : 0);
+    return xvals_bytes(fmt, K, MT) + (size_t)MT * (fmt == kFmtW4G64 ? (K / 64) * 8 : fmt == kFmtW4SB32 ? (K / 32) * 16 : 0);
 }
 
 // Stages x for one product and activation rows [m0, m0 + MT); run by one
@@ -127,56 +127,89 @@ __device__ __forceinline__ void stage_x_warp(const Item& it, int m0, int mrows, 
     constexpr bool kW4 = FMT != kFmtW8G16;
     const int hcpr = it.K >> 5, n = MT * hcpr;
     uint8_t* meta = xb + xvals_bytes(FMT, it.K, MT);
-    for (int i0 = lane; i0 < n; i0 += 64) {
-        uint4 v[2][4];
+    if constexpr (FMT == kFmtW4G64) {
+        // g64: one 64-value unit (a quantization group) per lane at a time;
+        // quad q of unit g of row m at (m * 8 + q) * G + g, record {z, f} at
+        // m * G + g, with z = 1032 * sum over even k + 72 * sum over odd k.
+        const int G = it.K >> 6, nu = MT * G;
+        for (int i = lane; i < nu; i += 32) {
+            const int m = i / G, g = i - m * G;
+            uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {               // both loads in flight before use
-            const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
+            for (int j = 0; j < 8; ++j) v[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (m < mrows) {
+                const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)g * 64);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[u][j] = make_uint4(0u, 0u, 0u, 0u);
-            if (i < n && m < mrows) {
-                const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)h * 32);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) v[u][j] = __ldg(src + j);
+                for (int j = 0; j < 8; ++j) v[j] = __ldg(src + j);
             }
+            uint32_t* w = reinterpret_cast<uint32_t*>(v);
+            uint32_t mb = 0u;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
+            const int e = mb != 0u ? min(126, max(-126, 14 - ((int)(mb >> 7) - 127))) : 0;
+            const float up = __int_as_float((e + 127) << 23), f = __int_as_float((127 - e) << 23);
+            float se = 0.0f, so = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
+                const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+                se = __fadd_rn(se, __half2float(a));
+                so = __fadd_rn(so, __half2float(b));
+                w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(xb) + (size_t)m * 8 * G + g;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[(size_t)q * G] = v[q];
+            reinterpret_cast<float2*>(meta)[(size_t)m * G + g] =
+                make_float2(__fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so)), f);
         }
+    } else {
+        for (int i0 = lane; i0 < n; i0 += 64) {
+            uint4 v[2][4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
-            if (i >= n) break;
-            uint32_t* w = reinterpret_cast<uint32_t*>(v[u]);
-            if constexpr (kW4) {
-                uint32_t mb = 0u;
+            for (int u = 0; u < 2; ++u) {               // both loads in flight before use
+                const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
-                const int e = mb != 0u ? min(126, max(-126, 14 - ((int)(mb >> 7) - 127))) : 0;
-                const float up = __int_as_float((e + 127) << 23), f = __int_as_float((127 - e) << 23);
-                float se = 0.0f, so = 0.0f;              // even-k and odd-k sums
+                for (int j = 0; j < 4; ++j) v[u][j] = make_uint4(0u, 0u, 0u, 0u);
+                if (i < n && m < mrows) {
+                    const uint4* src = reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)h * 32);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
-                    const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
-                    se = __fadd_rn(se, __half2float(a));
-                    so = __fadd_rn(so, __half2float(b));
-                    w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+                    for (int j = 0; j < 4; ++j) v[u][j] = __ldg(src + j);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(xb) + (size_t)m * 4 * hcpr + h;
+            }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[u][q];
-                if (FMT == kFmtW4G64) {
-                    const float z = __fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so));
-                    reinterpret_cast<float2*>(meta)[(size_t)m * hcpr + h] = make_float2(z, f);
-                } else {
-                    const float z = __fmaf_rn(1024.0f, se, __fmul_rn(64.0f, so));
+            for (int u = 0; u < 2; ++u) {
+                const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
+                if (i >= n) break;
+                uint32_t* w = reinterpret_cast<uint32_t*>(v[u]);
+                if constexpr (kW4) {
+                    uint32_t mb = 0u;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
+                    const int e = mb != 0u ? min(126, max(-126, 14 - ((int)(mb >> 7) - 127))) : 0;
+                    const float up = __int_as_float((e + 127) << 23), f = __int_as_float((127 - e) << 23);
+                    float se = 0.0f, so = 0.0f;              // even-k and odd-k sums
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
+                        const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+                        se = __fadd_rn(se, __half2float(a));
+                        so = __fadd_rn(so, __half2float(b));
+                        w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(xb) + (size_t)m * 4 * hcpr + h;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) dst[(size_t)q * hcpr] = v[u][q];
+                    const float z = __fmaf_rn(1024.0f, se, __fmul_rn(64.0f, so));   // sb32
                     reinterpret_cast<float4*>(meta)[(size_t)m * hcpr + h] =
                         make_float4(z, __fmul_rn(f, __fadd_rn(se, so)), f, 0.0f);
-                }
-            } else {
-                float4* dst = reinterpret_cast<float4*>(xb) + (size_t)m * 8 * hcpr + h;
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(xb) + (size_t)m * 8 * hcpr + h;
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    dst[(size_t)q * hcpr] = make_float4(bf16lo_f32(w[2 * q]), bf16hi_f32(w[2 * q]),
-                                                        bf16lo_f32(w[2 * q + 1]), bf16hi_f32(w[2 * q + 1]));
+                    for (int q = 0; q < 8; ++q)
+                        dst[(size_t)q * hcpr] = make_float4(bf16lo_f32(w[2 * q]), bf16hi_f32(w[2 * q]),
+                                                            bf16lo_f32(w[2 * q + 1]), bf16hi_f32(w[2 * q + 1]));
+                }
             }
         }
     }
@@ -204,63 +237,94 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
     // x quads: (m * Q + q) * hcpr + h, Q = 4 (bf16) or 8 (fp32) quads per half-chunk
     const uint32_t xstride = (uint32_t)hcpr * 16u;
     const uint32_t xa0 = x_s + (uint32_t)li * 16u;
-    constexpr uint32_t kMeta = FMT == kFmtW4G64 ? 8u : 16u;          // metadata record bytes
-    const uint32_t xm0 = x_s + (uint32_t)xvals_bytes(FMT, it.K, MT) + (uint32_t)li * kMeta;
+    const uint32_t xm0 = x_s + (uint32_t)xvals_bytes(FMT, it.K, MT) + (uint32_t)li * 16u;   // sb32 records
     float yacc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) yacc[r][m] = 0.0f;
 
-    if (kW4) {
-        // W4G64: codes at row * crb + h * 16, scale at (h / 2) * 2.
-        // W4SB32: record at row * crb + (h / 8) * 144; T is a multiple of 8
-        // (K % 256 == 0), so a lane always sees the same group j = li % 8.
-        const int j = li & 7;
+    if constexpr (FMT == kFmtW4G64) {
+        // One 64-weight group (unit) per lane and row: 32 code bytes at
+        // row * crb + unit * 32, its scale at unit * 2; x as 8 quads per unit
+        // (quad q of unit g at (m * 8 + q) * G + g) and a record {z, f}.
+        const int G = it.K >> 6;
+        const uint32_t gstride = (uint32_t)G * 16u;
+        const uint32_t xmg0 = x_s + (uint32_t)xvals_bytes(FMT, it.K, MT) + (uint32_t)li * 8u;
         uint32_t ca[RW], sa[RW];
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
-            if (FMT == kFmtW4G64) {
-                ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)li * 16u;
-                sa[r] = ssc_s + (uint32_t)(rbase + r) * srb + (uint32_t)(li >> 1) * 2u;
-            } else {
-                ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)(li >> 3) * 144u;
-                sa[r] = 0u;
-            }
+            ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)li * 32u;
+            sa[r] = ssc_s + (uint32_t)(rbase + r) * srb + (uint32_t)li * 2u;
         }
+        for (int hj = 0; hj < HJ; ++hj) {
+            const uint32_t du = (uint32_t)(hoff + hj) * (uint32_t)T;   // first unit of this step
+            float2 xm[MT];                               // {z, f}
+#pragma unroll
+            for (int m = 0; m < MT; ++m) xm[m] = lds64f_a(xmg0 + ((uint32_t)m * (uint32_t)G + du) * 8u);
+            uint4 c0[RW], c1[RW];
+            float sA[RW];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                c0[r] = lds128_a(ca[r] + du * 32u);
+                c1[r] = lds128_a(ca[r] + du * 32u + 16u);
+                sA[r] = __half2float(__ushort_as_half((unsigned short)lds16_a(sa[r] + du * 2u)));
+            }
+            // one accumulator for even k ((1024 + u) x), started at -z, and one
+            // for odd k ((1024 + 16 u) x) per row and m, whatever the launch
+            // shape, so a row's sums do not depend on RW or batching
+            float lo[RW][MT], hi[RW][MT];
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    lo[r][m] = -xm[m].x;
+                    hi[r][m] = 0.0f;
+                }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    const uint4 X = lds128_a(xa0 + du * 16u + (uint32_t)(m * 8 + q) * gstride);
+#pragma unroll
+                    for (int r = 0; r < RW; ++r)
+                        dot8_w4_f16(word_of(q < 4 ? c0[r] : c1[r], q & 3), X, lo[r][m], hi[r][m]);
+                }
+            }
+            // sum_k q_k x'_k = lo + hi / 16, back to x's scale with f = 2^-e_g
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+                    yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].y), __fmaf_rn(hi[r][m], 0.0625f, lo[r][m]),
+                                           yacc[r][m]);
+        }
+    } else if constexpr (kW4) {
+        // W4SB32: record at row * crb + (h / 8) * 144; T is a multiple of 8
+        // (K % 256 == 0), so a lane always sees the same group j = li % 8.
+        const int j = li & 7;
+        uint32_t ca[RW];
+#pragma unroll
+        for (int r = 0; r < RW; ++r) ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)(li >> 3) * 144u;
         for (int hj = 0; hj < HJ; hj += U) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (u > 0 && hj + u >= HJ) break;
                 const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
-                float4 xm[MT];                           // g64: {z, f}; sb32: {z, f * sum, f}
+                float4 xm[MT];                           // {z, f * sum, f}
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const uint32_t a = xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * kMeta;
-                    if (FMT == kFmtW4G64) {
-                        const float2 t = lds64f_a(a);
-                        xm[m] = make_float4(t.x, t.y, 0.0f, 0.0f);
-                    } else {
-                        xm[m] = lds128f_a(a);
-                    }
-                }
+                for (int m = 0; m < MT; ++m) xm[m] = lds128f_a(xm0 + ((uint32_t)m * (uint32_t)hcpr + dh) * 16u);
                 uint4 c[RW];
                 float sA[RW], sB[RW];
 #pragma unroll
                 for (int r = 0; r < RW; ++r) {
-                    if (FMT == kFmtW4G64) {
-                        c[r] = lds128_a(ca[r] + dh * 16u);
-                        sA[r] = __half2float(__ushort_as_half((unsigned short)lds16_a(sa[r] + dh)));
-                        sB[r] = 0.0f;
-                    } else {
-                        const uint32_t rec = ca[r] + (dh >> 3) * 144u;
-                        const uint4 hd = lds128_a(rec);
-                        c[r] = lds128_a(rec + 16u + (uint32_t)j * 16u);
-                        const float d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xffffu)));
-                        const float dm = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
-                        sA[r] = __fmul_rn(d, (float)sb_field(hd.y, hd.z, hd.w, 0, j));
-                        sB[r] = __fmul_rn(dm, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
-                    }
+                    const uint32_t rec = ca[r] + (dh >> 3) * 144u;
+                    const uint4 hd = lds128_a(rec);
+                    c[r] = lds128_a(rec + 16u + (uint32_t)j * 16u);
+                    const float d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xffffu)));
+                    const float dm = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
+                    sA[r] = __fmul_rn(d, (float)sb_field(hd.y, hd.z, hd.w, 0, j));
+                    sB[r] = __fmul_rn(dm, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
                 }
                 // one accumulator for even k ((1024 + u) x), started at -z, and
                 // one for odd k ((1024 + 16 u) x) per row and m, whatever the
@@ -282,19 +346,15 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                         for (int r = 0; r < RW; ++r) dot8_w4_f16(word_of(c[r], i), X, lo[r][m], hi[r][m]);
                     }
                 }
-                // sum_k q_k x'_k (g64) or sum_k u_k x'_k (sb32) = lo + hi / 16;
+                // sum_k u_k x'_k = lo + hi / 16;
                 // back to x's scale with f = 2^-e_h
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         const float a = __fmaf_rn(hi[r][m], 0.0625f, lo[r][m]);
-                        if (FMT == kFmtW4G64) {
-                            yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].y), a, yacc[r][m]);
-                        } else {
-                            yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].z), a, yacc[r][m]);
-                            yacc[r][m] = __fmaf_rn(-sB[r], xm[m].y, yacc[r][m]);
-                        }
+                        yacc[r][m] = __fmaf_rn(__fmul_rn(sA[r], xm[m].z), a, yacc[r][m]);
+                        yacc[r][m] = __fmaf_rn(-sB[r], xm[m].y, yacc[r][m]);
                     }
             }
         }
@@ -622,18 +682,22 @@ cudaError_t launch_one(const Batch<MAXI>& prm, size_t smem, int grid, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
-// Lane and warp layout of a product's rows: T lanes per team (a power of two
-// dividing K/32), KS warps per row (when T == 32, long rows are split so that
-// each warp covers about two half-chunks per lane), HJ half-chunks per lane.
+// Lane and warp layout of a product's rows. A lane's unit of a row is one
+// 64-weight group for g64 and a 32-weight half-chunk otherwise; T lanes per
+// team (a power of two dividing the units per row), KS warps per row (when
+// T == 32, long rows are split so that each warp keeps at least 128 weights
+// per lane and row), HJ units per lane and warp.
 struct Layout { int T, KS, HJ, teams; };
-Layout layout_of(int K) {
-    const int hcpr = K / 32;
+Layout layout_of(int fmt, int K) {
+    const int units = fmt == kFmtW4G64 ? K / 64 : K / 32;
+    const int min_hj = fmt == kFmtW4G64 ? 1 : 2;
     Layout l;
     l.T = 32;
-    while (l.T > 1 && (hcpr % l.T) != 0) l.T >>= 1;
-    const int hj_all = hcpr / l.T;
+    while (l.T > 1 && (units % l.T) != 0) l.T >>= 1;
+    const int hj_all = units / l.T;
     l.KS = 1;
-    while (l.T == 32 && kConsumerWarps % (l.KS * 2) == 0 && hj_all % (l.KS * 2) == 0 && hj_all / (l.KS * 2) >= 2)
+    while (l.T == 32 && kConsumerWarps % (l.KS * 2) == 0 && hj_all % (l.KS * 2) == 0 &&
+           hj_all / (l.KS * 2) >= min_hj)
         l.KS *= 2;
     l.HJ = hj_all / l.KS;
     l.teams = (kConsumerWarps / l.KS) * (32 / l.T);
@@ -646,7 +710,7 @@ Layout layout_of(int K) {
 #define RQ_GEMV_RW_MAX 4
 #endif
 int rw_allowed(int fmt, int K) {
-    const Layout l = layout_of(K);
+    const Layout l = layout_of(fmt, K);
     if (RQ_GEMV_RW_MAX < 4) return RQ_GEMV_RW_MAX;
     auto sb = [&](size_t R) { return round16(R * code_row_bytes(fmt, K)) + round16(R * scale_row_bytes(fmt, K)); };
     if (sb((size_t)l.teams * 4) <= 48 * 1024) return 4;
@@ -656,7 +720,7 @@ int rw_allowed(int fmt, int K) {
 // Per-item launch geometry for rows-per-team RW; false for a shape that does
 // not fit even with one staged-x buffer.
 bool plan_item(int fmt, int K, int N, int MT, int RW, Item& it, size_t& stage_b) {
-    const Layout l = layout_of(K);
+    const Layout l = layout_of(fmt, K);
     const size_t crb = code_row_bytes(fmt, K), srb = scale_row_bytes(fmt, K);
     int rho = 1;
     while (((size_t)rho * srb) % 16 != 0) rho <<= 1;     // srb is even, so rho <= 8

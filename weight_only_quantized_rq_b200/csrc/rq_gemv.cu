@@ -112,8 +112,9 @@ __host__ __device__ constexpr size_t xbuf_bytes(int fmt, int K, int MT) {
     return xvals_bytes(fmt, K, MT) + (size_t)MT * (fmt == kFmtW4G64 ? (K / 64) * 8 : fmt == kFmtW4SB32 ? (K / 32) * 16 : 0);
 }
 
-// Stages x for one product and activation rows [m0, m0 + MT); run by one
-// warp, lane i taking half-chunks i, i + 32, ...
+// Stages x for one product and activation rows [m0, m0 + MT); the calling
+// threads split it, thread `first` of `stride` taking units first,
+// first + stride, ... (a unit is 64 values for g64, 32 otherwise).
 //  int4 formats: fp16 quads in natural order (quad q = x[8q .. 8q+7]), each
 //  half-chunk h (32 values) scaled by the power of two 2^e_h that puts its
 //  largest |x| in [2^14, 2^15) (exact for every value no more than 2^32 times
@@ -122,8 +123,38 @@ __host__ __device__ constexpr size_t xbuf_bytes(int fmt, int K, int MT) {
 //  odd k; sb32: 1024 / 64), summed from the fp16 values the products use;
 //  g64 keeps {z, f}, sb32 {z, f * sum, f, 0}.
 //  int8 format: fp32 quads (quad q = x[4q .. 4q+3]).
+// First item whose cost range ends after lo (binary search: items are in
+// cost order), or count.
+template <int MAXI>
+__device__ __forceinline__ int item_after(const Batch<MAXI>& p, long long lo) {
+    int a = 0, b = p.count;
+    while (a < b) {
+        const int c = (a + b) >> 1;
+        if (p.it[c].cost1 <= lo) a = c + 1;
+        else b = c;
+    }
+    return a;
+}
+
+// Index of the first item with rows in the cost range [lo, hi), or -1.
+template <int MAXI>
+__device__ __forceinline__ int first_item(const Batch<MAXI>& p, long long lo, long long hi) {
+    for (int i = item_after(p, lo); i < p.count; ++i) {
+        const Item& it = p.it[i];
+        if (it.cost0 >= hi) break;
+        int ua, ub;
+        item_units(it, lo, hi, ua, ub);
+        if (ua * it.rho < min(ub * it.rho, it.N)) return i;
+    }
+    return -1;
+}
+
+// Named barriers: 1 .. kConsumerWarps (k-slice teams), kCoopBarrier (the
+// consumers and the stager after staging a CTA's first item).
+constexpr int kCoopBarrier = 15;
+
 template <int FMT, int MT>
-__device__ __forceinline__ void stage_x_warp(const Item& it, int m0, int mrows, uint8_t* xb, int lane) {
+__device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xb, int first, int stride) {
     constexpr bool kW4 = FMT != kFmtW8G16;
     const int hcpr = it.K >> 5, n = MT * hcpr;
     uint8_t* meta = xb + xvals_bytes(FMT, it.K, MT);
@@ -132,7 +163,7 @@ __device__ __forceinline__ void stage_x_warp(const Item& it, int m0, int mrows, 
         // quad q of unit g of row m at (m * 8 + q) * G + g, record {z, f} at
         // m * G + g, with z = 1032 * sum over even k + 72 * sum over odd k.
         const int G = it.K >> 6, nu = MT * G;
-        for (int i = lane; i < nu; i += 32) {
+        for (int i = first; i < nu; i += stride) {
             const int m = i / G, g = i - m * G;
             uint4 v[8];
 #pragma unroll
@@ -164,11 +195,11 @@ __device__ __forceinline__ void stage_x_warp(const Item& it, int m0, int mrows, 
                 make_float2(__fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so)), f);
         }
     } else {
-        for (int i0 = lane; i0 < n; i0 += 64) {
+        for (int i0 = first; i0 < n; i0 += 2 * stride) {
             uint4 v[2][4];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {               // both loads in flight before use
-                const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
+                const int i = i0 + stride * u, m = i / hcpr, h = i - m * hcpr;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) v[u][j] = make_uint4(0u, 0u, 0u, 0u);
                 if (i < n && m < mrows) {
@@ -179,7 +210,7 @@ __device__ __forceinline__ void stage_x_warp(const Item& it, int m0, int mrows, 
             }
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const int i = i0 + 32 * u, m = i / hcpr, h = i - m * hcpr;
+                const int i = i0 + stride * u, m = i / hcpr, h = i - m * hcpr;
                 if (i >= n) break;
                 uint32_t* w = reinterpret_cast<uint32_t*>(v[u]);
                 if constexpr (kW4) {
@@ -545,7 +576,7 @@ gemv_kernel(const Batch<MAXI> p) {
             const uint64_t pol = l2_evict_first_policy();
             int gi = 0;
             bool ok = true;
-            for (int i = 0; i < p.count && ok; ++i) {
+            for (int i = item_after(p, lo); i < p.count && ok; ++i) {
                 const Item& it = p.it[i];
                 if (it.cost0 >= hi) break;               // items are in cost order
                 if (it.cost1 <= lo) continue;            // no overlap: skip without dividing
@@ -573,10 +604,19 @@ gemv_kernel(const Batch<MAXI> p) {
         return;
     }
 
+    // A CTA's first item is staged by the consumer warps and the stager
+    // together (it is on the critical path of a dependent launch); the
+    // stager alone stages the later ones while the consumers compute.
+    const int i_first = first_item(p, lo, hi);
+    constexpr int kCoop = (kConsumerWarps + 1) * 32;
     if (warp == kStagerWarp) {                           // x of each item into alternating buffers
         grid_dep_wait();                                 // x is written by the previous kernel
-        int xi = 0;
-        for (int i = 0; i < p.count; ++i) {
+        if (i_first < 0) return;
+        stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, kConsumerWarps * 32 + lane, kCoop);
+        asm volatile("bar.sync %0, %1;" :: "n"(kCoopBarrier), "n"(kCoop) : "memory");
+        mbar_arrive(&xfull[0]);
+        int xi = 1;
+        for (int i = i_first + 1; i < p.count; ++i) {
             const Item& it = p.it[i];
             if (it.cost0 >= hi) break;
             if (it.cost1 <= lo) continue;
@@ -586,7 +626,7 @@ gemv_kernel(const Batch<MAXI> p) {
             const int b = xi % p.nxb;
             if (xi >= p.nxb && !mbar_wait_bounded(&xempty[b], ((xi / p.nxb) - 1) & 1, kStatusXWait, kStagerNapNs))
                 break;
-            stage_x_warp<FMT, MT>(it, p.m0, p.mrows, smem + p.x_off + (size_t)b * p.x_bytes, lane);
+            stage_x<FMT, MT>(it, p.m0, p.mrows, smem + p.x_off + (size_t)b * p.x_bytes, lane, 32);
             mbar_arrive(&xfull[b]);                      // each lane: its stores are released
             ++xi;
         }
@@ -595,7 +635,11 @@ gemv_kernel(const Batch<MAXI> p) {
 
     // ---- consumers ---------------------------------------------------------
     const uint32_t smem_s = smem_u32(smem);
-    grid_dep_wait();                                     // y may be read by the previous kernel
+    grid_dep_wait();                                     // x is written by the previous kernel
+    if (i_first >= 0) {
+        stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, tid, kCoop);
+        asm volatile("bar.sync %0, %1;" :: "n"(kCoopBarrier), "n"(kCoop) : "memory");
+    }
     RQ_PHASE_MARK(1);
     Ring ring;
     ring.full = full;
@@ -608,7 +652,7 @@ gemv_kernel(const Batch<MAXI> p) {
     ring.s = 0;
     ring.ph = 0u;
     int xi = 0;                                          // items done
-    for (int i = 0; i < p.count; ++i) {
+    for (int i = i_first < 0 ? p.count : i_first; i < p.count; ++i) {
         const Item it = p.it[i];                         // this item's fields in registers
         if (it.cost0 >= hi) break;                       // items are in cost order
         if (it.cost1 <= lo) continue;                    // no overlap: skip without dividing

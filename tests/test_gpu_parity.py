@@ -192,6 +192,18 @@ WGEMM_CASES = [
     ("w4sb32", 2560, 99, 8),
     ("w4sb32", 256, 7, 32),
     ("w4sb32", 768, 33, 3),
+    # M >= 33: int4 g64 and int8 g16 on the tensor-core prefill kernel
+    ("w4g64", 2048, 300, 33),
+    ("w4g64", 4096, 257, 64),
+    ("w4g64", 768, 130, 100),
+    ("w4g64", 64, 5, 128),
+    ("w4g64", 320, 77, 48),
+    ("w4g64", 16384, 40, 128),
+    ("w8g16", 4096, 200, 64),
+    ("w8g16", 2048, 129, 128),
+    ("w8g16", 448, 33, 80),
+    # the superblock format stays on the GEMV kernel at every M
+    ("w4sb32", 512, 40, 64),
 ]
 
 
@@ -209,7 +221,7 @@ def test_wgemm_matches_oracle(case):
 
 
 @pytest.mark.parametrize("fmt,unit", [("w4g64", 2.0 ** -6), ("w8g16", 2.0 ** -10)])
-@pytest.mark.parametrize("M", [1, 3, 8])
+@pytest.mark.parametrize("M", [1, 3, 8, 64, 128])
 def test_wgemm_exact_integer_products(fmt, unit, M):
     """w = q 2^-e and small-integer x: every partial sum is an integer
     multiple of 2^-e below 2^24, so the fp32 result must be exact."""
@@ -299,6 +311,8 @@ def test_full_size_workloads_sampled(widx):
     ("w4g64", [(1024, 300), (1024, 64), (4096, 77)], 2),
     ("w8g16", [(2048, 130), (4096, 33), (448, 9)], 1),
     ("w4sb32", [(2560, 200), (10240, 40), (256, 3)], 3),
+    ("w4g64", [(2048, 300), (4096, 129), (64, 7)], 64),
+    ("w8g16", [(1024, 257), (448, 5)], 128),
 ])
 def test_wgemm_batch_matches_oracle(fmt, shapes, M):
     """One launch over products of different shapes equals the oracle per

@@ -100,7 +100,9 @@ int rq_wgemm(const void* x, int M, int K, int N, const rq_packed* w, float* y, v
     if (s != RQ_OK) return s;
     if (!aligned16(x) || !aligned16(y)) return RQ_ERR_MISALIGNED;
     rq::WgemmArgs a = {w->fmt, M, K, N, x, w->codes, w->scales, y};
-    return cuda_status(rq::launch_gemv(&a, 1, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rq::prefill_supported(w->fmt, M)) return cuda_status(rq::launch_prefill(a, st));
+    return cuda_status(rq::launch_gemv(&a, 1, st));
 }
 
 int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
@@ -116,7 +118,15 @@ int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
         if (!aligned16(it.x) || !aligned16(it.y)) return RQ_ERR_MISALIGNED;
         a[i] = {it.w->fmt, M, it.w->K, it.w->N, it.x, it.w->codes, it.w->scales, it.y};
     }
-    return cuda_status(rq::launch_gemv(a, count, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rq::prefill_supported(a[0].fmt, M)) {            // compute-bound: one tensor-core launch per product
+        for (int i = 0; i < count; ++i) {
+            const int s = cuda_status(rq::launch_prefill(a[i], st));
+            if (s != RQ_OK) return s;
+        }
+        return RQ_OK;
+    }
+    return cuda_status(rq::launch_gemv(a, count, st));
 }
 
 int rq_dequant(const rq_packed* w, float* W_out, void* stream) {
@@ -146,10 +156,11 @@ int rq_last_cuda_error(void) { return t_last_cuda; }
 int rq_device_status(void* stream, int* word) {
     if (!word) return RQ_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    unsigned a = 0, b = 0;
+    unsigned a = 0, b = 0, c = 0;
     int s = cuda_status(rq::status_pack(st, &a));
     if (s == RQ_OK) s = cuda_status(rq::status_gemv(st, &b));
-    *word = (int)(a | b);
+    if (s == RQ_OK) s = cuda_status(rq::status_prefill(st, &c));
+    *word = (int)(a | b | c);
     if (s != RQ_OK) return s;
     return *word ? RQ_ERR_DEVICE_TIMEOUT : RQ_OK;
 }

@@ -204,6 +204,12 @@ WGEMM_CASES = [
     ("w8g16", 448, 33, 80),
     # the superblock format stays on the GEMV kernel at every M
     ("w4sb32", 512, 40, 64),
+    # more tiles than SMs: persistent CTAs take two tiles (double-buffered accumulator)
+    ("w4g64", 512, 20000, 16),
+    ("w8g16", 256, 19500, 8),
+    # K split over a cluster with a half stage at the end of K (int4 scale windows)
+    ("w4g64", 832, 200, 24),
+    ("w8g16", 832, 130, 40),
 ]
 
 
@@ -313,6 +319,8 @@ def test_full_size_workloads_sampled(widx):
     ("w4sb32", [(2560, 200), (10240, 40), (256, 3)], 3),
     ("w4g64", [(2048, 300), (4096, 129), (64, 7)], 64),
     ("w8g16", [(1024, 257), (448, 5)], 128),
+    ("w4g64", [(512, 9000), (1024, 12000), (320, 3)], 32),
+    ("w8g16", [(256, 4000), (512, 300), (2048, 16000)], 4),
 ])
 def test_wgemm_batch_matches_oracle(fmt, shapes, M):
     """One launch over products of different shapes equals the oracle per

@@ -101,7 +101,7 @@ int rq_wgemm(const void* x, int M, int K, int N, const rq_packed* w, float* y, v
     if (!aligned16(x) || !aligned16(y)) return RQ_ERR_MISALIGNED;
     rq::WgemmArgs a = {w->fmt, M, K, N, x, w->codes, w->scales, y};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (rq::prefill_supported(w->fmt, M)) return cuda_status(rq::launch_prefill(a, st));
+    if (rq::tc_supported(w->fmt, M)) return cuda_status(rq::launch_tc(&a, 1, st));
     return cuda_status(rq::launch_gemv(&a, 1, st));
 }
 
@@ -119,13 +119,7 @@ int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
         a[i] = {it.w->fmt, M, it.w->K, it.w->N, it.x, it.w->codes, it.w->scales, it.y};
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (rq::prefill_supported(a[0].fmt, M)) {            // compute-bound: one tensor-core launch per product
-        for (int i = 0; i < count; ++i) {
-            const int s = cuda_status(rq::launch_prefill(a[i], st));
-            if (s != RQ_OK) return s;
-        }
-        return RQ_OK;
-    }
+    if (rq::tc_supported(a[0].fmt, M)) return cuda_status(rq::launch_tc(a, count, st));
     return cuda_status(rq::launch_gemv(a, count, st));
 }
 
@@ -159,7 +153,7 @@ int rq_device_status(void* stream, int* word) {
     unsigned a = 0, b = 0, c = 0;
     int s = cuda_status(rq::status_pack(st, &a));
     if (s == RQ_OK) s = cuda_status(rq::status_gemv(st, &b));
-    if (s == RQ_OK) s = cuda_status(rq::status_prefill(st, &c));
+    if (s == RQ_OK) s = cuda_status(rq::status_tc(st, &c));
     *word = (int)(a | b | c);
     if (s != RQ_OK) return s;
     return *word ? RQ_ERR_DEVICE_TIMEOUT : RQ_OK;

@@ -51,16 +51,17 @@ struct WgemmArgs {
 constexpr int kMaxBatch = 160;
 cudaError_t launch_gemv(const WgemmArgs* a, int count, cudaStream_t st);
 
-// Compute-bound path (prefill, kPrefillMinM <= M <= 128; int4 g64 and int8
-// g16): bf16 tiles dequantized into shared memory, tcgen05.mma into TMEM.
-constexpr int kPrefillMinM = 33;
-bool prefill_supported(int fmt, int M);
-cudaError_t launch_prefill(const WgemmArgs& a, cudaStream_t st);
+// Tensor-core path (kTcMinM <= M <= 128; int4 g64 and int8 g16): bf16 tiles
+// dequantized into tensor memory, tcgen05.mma against x in shared memory.
+// `count` independent products of one format and one M share a launch.
+constexpr int kTcMinM = 3;
+bool tc_supported(int fmt, int M);
+cudaError_t launch_tc(const WgemmArgs* a, int count, cudaStream_t st);
 
 // Read and clear the device status word of each kernel file (synchronizes st).
 cudaError_t status_pack(cudaStream_t st, unsigned* word);
 cudaError_t status_gemv(cudaStream_t st, unsigned* word);
-cudaError_t status_prefill(cudaStream_t st, unsigned* word);
+cudaError_t status_tc(cudaStream_t st, unsigned* word);
 
 int sm_count();   // multiprocessors of the current device
 

@@ -45,6 +45,16 @@ def peaks():
         return HBM_FALLBACK, "fallback"
 
 
+def tensor_peak():
+    """Dense bf16 tensor throughput (TFLOP/s) for a kernel timed in a short
+    burst: the measured one when available."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -197,10 +207,78 @@ def recorded_traffic(kernel: str):
 
 
 # -------------------------------------------------------------- ours ------
-def run_ours(args, w, M):
+def pack_workload(w, dev):
+    """Quantize-pack every matrix of a workload on the GPU (not timed)."""
     import torch
     import weight_only_quantized_rq_b200 as rq
     from weight_only_quantized_rq_b200 import workloads as wl
+    mats = []
+    for j, layer, m in w.matrices():
+        W = wl.weights(w, j, m, device=str(dev))
+        a = torch.from_numpy(wl.act_sq(w, m.K)).to(dev) if m.n_cand > 1 else None
+        p = rq.rq_quantize_pack(W, m.fmt, a, m.n_cand, 0.7 if m.n_cand > 1 else 1.0, 1.0)
+        mats.append((j, m, p))
+        del W
+    torch.cuda.synchronize()
+    return mats
+
+
+class Problem:
+    """One M over a packed workload: every product's x in one device block,
+    every y in another, and the step as batched launches (one per format and
+    chunk of at most 160 products; the products are independent)."""
+
+    def __init__(self, w, mats, M, dev):
+        import torch
+        import weight_only_quantized_rq_b200 as rq
+        from weight_only_quantized_rq_b200 import workloads as wl
+        self.M = M
+        xs_elems = sum(M * m.K + 8 for _, m, _ in mats)
+        ys_elems = sum(M * m.N + 4 for _, m, _ in mats)
+        self.xdev = torch.empty(xs_elems, dtype=torch.bfloat16, device=dev)
+        self.ydev = torch.empty(ys_elems, dtype=torch.float32, device=dev)
+        self.calls, xo, yo = [], 0, 0
+        for j, m, p in mats:
+            x = self.xdev[xo:xo + M * m.K].view(M, m.K)
+            x.copy_(wl.activations(w, j, m.K, M, device=str(dev)))
+            y = self.ydev[yo:yo + M * m.N].view(M, m.N)
+            self.calls.append((x, p, y, m))
+            xo += (M * m.K + 7) // 8 * 8
+            yo += (M * m.N + 3) // 4 * 4
+        self.packed_bytes = sum(p.nbytes for _, _, p in mats)
+        self.alg_bytes = sum(p.nbytes + 2 * M * p.K + 4 * M * p.N for _, _, p in mats)
+        self.flops = sum(2 * M * p.K * p.N for _, _, p in mats)
+        self.h2d = sum(M * m.K * 2 for _, m, _ in mats)
+        self.d2h = sum(M * m.N * 4 for _, m, _ in mats)
+        self.batches = []
+        self.kernel_launches = 0     # launches the library issues per step
+        for fmt in sorted({m.fmt for *_, m in self.calls}):
+            cs = [c for c in self.calls if c[3].fmt == fmt]
+            for i in range(0, len(cs), rq.MAX_BATCH):
+                ch = cs[i:i + rq.MAX_BATCH]
+                self.batches.append(rq.WgemmBatch([c[0] for c in ch], [c[1] for c in ch], [c[2] for c in ch]))
+                tc = M >= rq.TC_MIN_M and fmt in ("w4g64", "w8g16")
+                self.kernel_launches += -(-len(ch) // rq.TC_MAX_ITEMS) if tc else 1
+        torch.cuda.synchronize()
+
+    def step(self, stream):
+        for b in self.batches:
+            b(stream=stream)
+
+    def roofline_s(self, hbm_gbs, tflops):
+        """Lower bound on the step time: per product, the slower of its
+        weight/x/y traffic at the HBM rate and its flops at the tensor rate."""
+        t = 0.0
+        for x, p, y, m in self.calls:
+            b = p.nbytes + 2 * self.M * p.K + 4 * self.M * p.N
+            f = 2 * self.M * p.K * p.N
+            t += max(b / (hbm_gbs * 1e9), f / (tflops * 1e12))
+        return t
+
+
+def run_ours(args, w, M):
+    import torch
+    import weight_only_quantized_rq_b200 as rq
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -216,41 +294,13 @@ def run_ours(args, w, M):
         v, desc, thr, _ = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": round(v, 4), "unit": "GB/s", "cores": thr, "kind": "oracle", "sample": desc}
 
-    # pack the workload (not timed)
-    mats = []
-    for j, layer, m in w.matrices():
-        W = wl.weights(w, j, m, device=str(dev))
-        a = torch.from_numpy(wl.act_sq(w, m.K)).to(dev) if m.n_cand > 1 else None
-        p = rq.rq_quantize_pack(W, m.fmt, a, m.n_cand, 0.7 if m.n_cand > 1 else 1.0, 1.0)
-        mats.append((m, p))
-        del W
-    torch.cuda.synchronize()
-    # inputs: one device block holding every matrix's x, one for every y
-    xs_elems = sum(M * m.K for m, _ in mats)
-    ys_elems = sum(M * m.N for m, _ in mats)
-    xdev = torch.empty(xs_elems + 8 * len(mats), dtype=torch.bfloat16, device=dev)
-    ydev = torch.empty(ys_elems + 4 * len(mats), dtype=torch.float32, device=dev)
-    calls, xo, yo = [], 0, 0
-    for (m, p), (j, _, _) in zip(mats, w.matrices()):
-        x = xdev[xo:xo + M * m.K].view(M, m.K)
-        x.copy_(wl.activations(w, j, m.K, M, device=str(dev)))
-        y = ydev[yo:yo + M * m.N].view(M, m.N)
-        calls.append((x, p, y))
-        xo += (M * m.K + 7) // 8 * 8
-        yo += (M * m.N + 3) // 4 * 4
-    packed_bytes = sum(p.nbytes for _, p in mats)
-    alg_bytes = sum(p.nbytes + 2 * M * p.K + 4 * M * p.N for _, p in mats)
-    torch.cuda.synchronize()
-
+    mats = pack_workload(w, dev)
+    prob = Problem(w, mats, M, dev)
+    calls, packed_bytes, alg_bytes = prob.calls, prob.packed_bytes, prob.alg_bytes
     stream = torch.cuda.Stream(device=dev)
-    # the step: every product of the layer set in one rq_wgemm_batch launch
-    # (the products' inputs are independent); at most 160 items per launch
-    batches = [rq.WgemmBatch([c[0] for c in calls[i:i + rq.MAX_BATCH]], [c[1] for c in calls[i:i + rq.MAX_BATCH]],
-                             [c[2] for c in calls[i:i + rq.MAX_BATCH]]) for i in range(0, len(calls), rq.MAX_BATCH)]
 
     def step():
-        for b in batches:
-            b(stream=stream)
+        prob.step(stream)
 
     # the decode chain of a real token: per layer, the independent r/k/v
     # projections in one launch, then o, ffn key, ffn value, each depending on
@@ -273,6 +323,8 @@ def run_ours(args, w, M):
             else:
                 rq.rq_wgemm(part[0], part[1], part[2], stream=stream)
 
+    graphs = []
+
     def capture(fn):
         with torch.cuda.stream(stream):
             fn()
@@ -283,6 +335,7 @@ def run_ours(args, w, M):
             with torch.cuda.graph(g, stream=stream):
                 fn()
         torch.cuda.synchronize()
+        graphs.append(g)
         return g.replay
 
     run = capture(step)
@@ -323,45 +376,84 @@ def run_ours(args, w, M):
     chain_val = ws * packed_bytes / (ms_chain * 1e-3) / 1e9
 
     # end to end through the public API: pinned host x in, host y out
-    xh = torch.empty(xdev.shape, dtype=xdev.dtype, pin_memory=True)
-    yh = torch.empty(ydev.shape, dtype=ydev.dtype, pin_memory=True)
-    xh.copy_(xdev)
-    h2d = sum(M * m.K * 2 for m, _ in mats)
-    d2h = sum(M * m.N * 4 for m, _ in mats)
+    xh = torch.empty(prob.xdev.shape, dtype=prob.xdev.dtype, pin_memory=True)
+    yh = torch.empty(prob.ydev.shape, dtype=prob.ydev.dtype, pin_memory=True)
+    xh.copy_(prob.xdev)
 
     def e2e_step():
-        xdev.copy_(xh, non_blocking=True)
+        prob.xdev.copy_(xh, non_blocking=True)
         run()
-        yh.copy_(ydev, non_blocking=True)
+        yh.copy_(prob.ydev, non_blocking=True)
 
     ms_e2e = timed(e2e_step, args.steps)
     e2e_val = ws * packed_bytes / (ms_e2e * 1e-3) / 1e9
-    launches = len(batches)
-    status = rq.rq_device_status(stream)
+    launches = prob.kernel_launches
     hbm, src = peaks()
+    tc_peak, tc_src = tensor_peak()
     per_launch_bytes = alg_bytes / launches
     per_launch_s = ms_max * 1e-3 / launches
     achieved = per_launch_bytes / per_launch_s / 1e9
     traffic = recorded_traffic("gemv_batch_w4g64_m1")
+
+    # the same workload at the other activation-row counts of its config (the
+    # tensor-core path for M >= 3), and prefill on the 7.2B shapes
+    extra_m = [] if args.quick else [m for m in w.Ms if m != M]
+    small = {}
+    for m2 in extra_m:
+        pr = Problem(w, mats, m2, dev)
+        f = capture(lambda pr=pr: pr.step(stream))
+        ms2 = timed(f, args.steps)
+        small[str(m2)] = {"ms_per_step": round(ms2, 5), "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
+                          "pct_hbm_measured": round(100 * pr.packed_bytes / (ms2 * 1e-3) / 1e9 / hbm, 2),
+                          "roofline_frac": round(pr.roofline_s(hbm, tc_peak) / (ms2 * 1e-3), 4),
+                          "launches_per_step": pr.kernel_launches,
+                          "kernel": "gemv_kernel" if m2 <= 2 else "tc_kernel (tcgen05, A in tensor memory)"}
+        del pr
+    prefill = None
+    if not args.quick:
+        from weight_only_quantized_rq_b200 import workloads as wl
+        wp = wl.WORKLOADS[4]
+        mats_p = pack_workload(wp, dev)
+        prefill = {"workload": wp.name}
+        for m2 in (64, 128):
+            pr = Problem(wp, mats_p, m2, dev)
+            f = capture(lambda pr=pr: pr.step(stream))
+            ms2 = timed(f, args.steps)
+            t_roof = pr.roofline_s(hbm, tc_peak)
+            prefill[str(m2)] = {"ms_per_step": round(ms2, 5),
+                                "TFLOP_s": round(ws * pr.flops / (ms2 * 1e-3) / 1e12, 2),
+                                "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
+                                "pct_bf16_peak_measured": round(100 * pr.flops / (ms2 * 1e-3) / 1e12 / tc_peak, 2),
+                                "roofline": {"bound": "max(tensor, hbm) per product", "time_s": t_roof,
+                                             "frac": round(t_roof / (ms2 * 1e-3), 4), "tensor_peak_tflops": tc_peak,
+                                             "hbm_peak_gbs": hbm, "peak_source": tc_src},
+                                "launches_per_step": pr.kernel_launches}
+            del pr
+        del mats_p
+    status = rq.rq_device_status(stream)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {**config_of(w, M), "packed_bytes_per_step": packed_bytes, "step": "one rq_wgemm_batch launch "
-                   "over the layer set's independent products", "graph": not args.no_graph, "pdl": True,
+        "config": {**config_of(w, M), "packed_bytes_per_step": packed_bytes, "step": "batched rq_wgemm_batch "
+                   "launches over the layer set's independent products", "graph": not args.no_graph, "pdl": True,
                    "parallelism": f"replicas{ws}" if ws > 1 else "single",
                    "pct_hbm_measured": round(100 * value / ws / hbm, 2),
                    "pct_hbm_nominal_8TBs": round(100 * value / ws / NOMINAL_HBM, 2)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": traffic,
-                     "kernel": "gemv_kernel<w4g64, M=1> (batched launch)", "peak_source": src,
+                     "kernel": "gemv_kernel<w4g64, M=1> (batched launch)" if M <= 2 else "tc_kernel",
+                     "peak_source": src,
                      "note": "algorithmic bytes (packed weights + x + y) per launch / CUDA-event time per launch"},
         "decode_chain": {"value": round(chain_val, 2), "unit": "GB/s", "ms_per_step": round(ms_chain, 5),
                          "launches_per_step": len(chain_parts),
                          "structure": "per layer: r/k/v in one batched launch, then o, ffn key, ffn value, "
                                       "each dependent on the previous launch"},
+        "small_m": small,
+        "prefill": prefill,
         "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": prob.h2d,
+                "d2h_bytes_per_step": prob.d2h},
         "gpu_launches": launches * args.steps,
         "clocks": clk,
         "device_status": status,
@@ -371,6 +463,7 @@ def run_ours(args, w, M):
     if ws > 1:
         import torch.distributed as dist
         del run, run_chain
+        graphs.clear()
         dist.destroy_process_group()
     return 0
 
@@ -386,6 +479,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--quick", action="store_true", help="headline line only (no other M, no prefill)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     from weight_only_quantized_rq_b200 import workloads as wl

@@ -37,6 +37,8 @@ FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_AS
 EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_dequant",
            "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
 MAX_BATCH = 160
+TC_MIN_M = 3         # activation rows from which int4 g64 / int8 g16 products run on the tensor cores
+TC_MAX_ITEMS = 96    # products per tensor-core launch (larger batches take several)
 
 
 class RqSearch(ctypes.Structure):

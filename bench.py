@@ -395,41 +395,37 @@ def run_ours(args, w, M):
     achieved = per_launch_bytes / per_launch_s / 1e9
     traffic = recorded_traffic("gemv_batch_w4g64_m1")
 
-    # the same workload at the other activation-row counts of its config (the
-    # tensor-core path for M >= 3), and prefill on the 7.2B shapes
-    extra_m = [] if args.quick else [m for m in w.Ms if m != M]
-    small = {}
-    for m2 in extra_m:
-        pr = Problem(w, mats, m2, dev)
-        f = capture(lambda pr=pr: pr.step(stream))
-        ms2 = timed(f, args.steps)
-        small[str(m2)] = {"ms_per_step": round(ms2, 5), "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
-                          "pct_hbm_measured": round(100 * pr.packed_bytes / (ms2 * 1e-3) / 1e9 / hbm, 2),
-                          "roofline_frac": round(pr.roofline_s(hbm, tc_peak) / (ms2 * 1e-3), 4),
-                          "launches_per_step": pr.kernel_launches,
-                          "kernel": "gemv_kernel" if m2 <= 2 else "tc_kernel (tcgen05, A in tensor memory)"}
-        del pr
-    prefill = None
+    # every configuration at each of its activation-row counts (the headline
+    # workload at its other M, and the other four configurations), one
+    # batched step per (configuration, M)
+    from weight_only_quantized_rq_b200 import workloads as wl
+    configs = {}
     if not args.quick:
-        from weight_only_quantized_rq_b200 import workloads as wl
-        wp = wl.WORKLOADS[4]
-        mats_p = pack_workload(wp, dev)
-        prefill = {"workload": wp.name}
-        for m2 in (64, 128):
-            pr = Problem(wp, mats_p, m2, dev)
-            f = capture(lambda pr=pr: pr.step(stream))
-            ms2 = timed(f, args.steps)
-            t_roof = pr.roofline_s(hbm, tc_peak)
-            prefill[str(m2)] = {"ms_per_step": round(ms2, 5),
-                                "TFLOP_s": round(ws * pr.flops / (ms2 * 1e-3) / 1e12, 2),
-                                "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
-                                "pct_bf16_peak_measured": round(100 * pr.flops / (ms2 * 1e-3) / 1e12 / tc_peak, 2),
-                                "roofline": {"bound": "max(tensor, hbm) per product", "time_s": t_roof,
-                                             "frac": round(t_roof / (ms2 * 1e-3), 4), "tensor_peak_tflops": tc_peak,
-                                             "hbm_peak_gbs": hbm, "peak_source": tc_src},
-                                "launches_per_step": pr.kernel_launches}
-            del pr
-        del mats_p
+        for wi, w2 in enumerate(wl.WORKLOADS):
+            Ms = [m for m in w2.Ms if not (w2 is w and m == M)]
+            if not Ms:
+                continue
+            mats2 = mats if w2 is w else pack_workload(w2, dev)
+            entry = {"workload": w2.name, "packed_bytes_per_step": sum(p.nbytes for _, _, p in mats2)}
+            for m2 in Ms:
+                pr = Problem(w2, mats2, m2, dev)
+                f = capture(lambda pr=pr: pr.step(stream))
+                ms2 = timed(f, min(args.steps, 10))
+                t_roof = pr.roofline_s(hbm, tc_peak)
+                entry[str(m2)] = {
+                    "ms_per_step": round(ms2, 5),
+                    "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
+                    "pct_hbm_measured": round(100 * pr.packed_bytes / (ms2 * 1e-3) / 1e9 / hbm, 2),
+                    "TFLOP_s": round(ws * pr.flops / (ms2 * 1e-3) / 1e12, 2),
+                    "pct_bf16_peak_measured": round(100 * pr.flops / (ms2 * 1e-3) / 1e12 / tc_peak, 2),
+                    "roofline_frac": round(t_roof / (ms2 * 1e-3), 4),
+                    "launches_per_step": pr.kernel_launches,
+                    "kernel": "gemv_kernel" if m2 < rq.TC_MIN_M else "tc_kernel"}
+                del pr
+            configs[f"config{wi + 1}"] = entry
+            if w2 is not w:
+                del mats2
+                torch.cuda.empty_cache()
     status = rq.rq_device_status(stream)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
@@ -449,8 +445,10 @@ def run_ours(args, w, M):
                          "launches_per_step": len(chain_parts),
                          "structure": "per layer: r/k/v in one batched launch, then o, ffn key, ffn value, "
                                       "each dependent on the previous launch"},
-        "small_m": small,
-        "prefill": prefill,
+        "configs": configs,
+        "configs_note": "per (configuration, M): one graph-captured step of batched launches over the "
+                        "configuration's products; roofline_frac = sum over products of max(bytes / HBM peak, "
+                        "flops / bf16 peak) divided by the step time",
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": prob.h2d,
                 "d2h_bytes_per_step": prob.d2h},
@@ -479,7 +477,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--quick", action="store_true", help="headline line only (no other M, no prefill)")
+    ap.add_argument("--quick", action="store_true", help="headline line only (no other configurations)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     from weight_only_quantized_rq_b200 import workloads as wl

@@ -202,8 +202,10 @@ WGEMM_CASES = [
     ("w8g16", 4096, 200, 64),
     ("w8g16", 2048, 129, 128),
     ("w8g16", 448, 33, 80),
-    # the superblock format stays on the GEMV kernel at every M
+    # superblock records on the tensor-core kernel (M >= 3)
     ("w4sb32", 512, 40, 64),
+    ("w4sb32", 2560, 300, 16),
+    ("w4sb32", 10240, 130, 128),
     # more tiles than SMs: persistent CTAs take two tiles (double-buffered accumulator)
     ("w4g64", 512, 20000, 16),
     ("w8g16", 256, 19500, 8),
@@ -245,8 +247,11 @@ def test_wgemm_exact_integer_products(fmt, unit, M):
 
 
 def test_wgemm_exact_superblock():
+    """Superblock weights c (q - 8) 2^-12 need up to 9 significant bits: exact
+    in the fp32 GEMV path (M <= 2); the tensor-core path (M >= 3) rounds w_hat
+    to bf16 and is covered by the tolerance cases."""
     rng = np.random.default_rng(23)
-    N, K, M = 50, 1024, 4
+    N, K, M = 50, 1024, 2
     q = rng.integers(0, 16, size=(N, K))
     qg = q.reshape(N, K // 32, 32)
     qg[:, :, 0], qg[:, :, 1] = 0, 15
@@ -317,6 +322,7 @@ def test_full_size_workloads_sampled(widx):
     ("w4g64", [(1024, 300), (1024, 64), (4096, 77)], 2),
     ("w8g16", [(2048, 130), (4096, 33), (448, 9)], 1),
     ("w4sb32", [(2560, 200), (10240, 40), (256, 3)], 3),
+    ("w4sb32", [(2560, 2560), (2560, 1000), (10240, 77)], 32),
     ("w4g64", [(2048, 300), (4096, 129), (64, 7)], 64),
     ("w8g16", [(1024, 257), (448, 5)], 128),
     ("w4g64", [(512, 9000), (1024, 12000), (320, 3)], 32),

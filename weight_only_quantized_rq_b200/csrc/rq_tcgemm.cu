@@ -1,6 +1,7 @@
 // rq_tcgemm.cu -- y = x * w_hat^T on the 5th-generation tensor cores, for
 // activation blocks of 3 <= M <= 128 rows (small-M decode batches and
-// prefill), int4 group-64 and int8 group-16 formats.
+// prefill), for all three formats: int4 group-64, int8 group-16 and the int4
+// asymmetric superblock (144-byte records of 8 groups of 32).
 //
 // Sources: RWKV-7 G1 1.5B int4 model card, summary paragraph (a tensor-core
 // GEMM beside the int4 GEMV and small-M kernels; output bit-identical to the
@@ -48,7 +49,13 @@
 //    nibble; fma.rn.f32.f16 against the fp16 scale and an exact fp32 offset
 //    gives q * s exactly; cvt.rn.bf16x2.f32 rounds each pair to bf16 in natural
 //    k order (one rounding per weight). int8: a byte permute gives fp16
-//    (1024 + u), the same FMA gives q * s.
+//    (1024 + u), the same FMA gives q * s. Superblock: each 256-K stage holds
+//    one 144-byte record per row (box rows of 144 bytes, unswizzled: the row
+//    stride of nine 16-byte chunks keeps 8 consecutive rows on distinct bank
+//    groups); a thread reads the record header and its two 32-weight groups,
+//    forms S = d * sc and M = dmin * m in fp32, places nibbles under an fp32
+//    exponent (128 + u) with a byte permute and evaluates S u - M with one FFMA
+//    before the bf16 rounding.
 //  * Work: a persistent CTA per SM walks the tiles of all products of the
 //    launch (largest K first). A single product with fewer tiles than about
 //    half the SMs is split along K over a thread-block cluster; the partial
@@ -261,7 +268,9 @@ __device__ __forceinline__ uint32_t lop_mask_or(uint32_t v, uint32_t m, uint32_t
 // (chunk c ^ (r % 8)), rows of 64 bytes the 64-byte pattern (c ^ (r / 2 % 4)).
 template <int RB>
 __device__ __forceinline__ uint32_t code_pos(int r, int c) {
-    return RB == 128 ? (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)) : (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    return RB == 128 ? (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4))
+         : RB == 64 ? (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4))
+                    : (uint32_t)(r * RB + (c << 4));                       // superblock records: unswizzled
 }
 
 // 8 NW int4 weights (NW code words, one fp16 scale) -> 4 NW bf16 pairs in
@@ -304,6 +313,33 @@ __device__ __forceinline__ void dq_w8(const uint4 (&c)[2], uint32_t sc, uint32_t
             const uint32_t e0 = prmt(w[i], 0x6464u, 0x4140u), e1 = prmt(w[i], 0x6464u, 0x4342u);
             o[8 * g + 2 * i] = pack_bf16(fma_h<0>(e0, sb, cf), fma_h<1>(e0, sb, cf));
             o[8 * g + 2 * i + 1] = pack_bf16(fma_h<0>(e1, sb, cf), fma_h<1>(e1, sb, cf));
+        }
+    }
+}
+
+// 64 superblock weights: groups 2h and 2h+1 of a 144-byte record (header
+// hd = fp16 d, fp16 dmin, 96-bit string of 6-bit sc_j / m_j; c0, c1 = the
+// groups' 16 code bytes each) -> 32 bf16 pairs. w = S u - M with S = d sc_j,
+// M = dmin m_j (both exact in fp32); u from the nibble under the fp32 exponent
+// of 128: (128 + u) S + (-128 S - M), then one rounding to bf16.
+__device__ __forceinline__ void dq_sb32(const uint4 hd, const uint4 c0, const uint4 c1, int h, uint32_t (&o)[32]) {
+    const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
+    const float dmin = __half2float(__ushort_as_half((uint16_t)(hd.x >> 16)));
+#pragma unroll
+    for (int gl = 0; gl < 2; ++gl) {
+        const int j = 2 * h + gl;
+        const float S = __fmul_rn(d, (float)sb_field(hd.y, hd.z, hd.w, 0, j));
+        const float Mv = __fmul_rn(dmin, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
+        const float c = __fsub_rn(__fmul_rn(-128.0f, S), Mv);
+        const uint4 cw = gl == 0 ? c0 : c1;
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float f[8];
+            unpack_w4(w[i], f);            // f[0..3]: k = 0, 2, 4, 6; f[4..7]: k = 1, 3, 5, 7 (128 + u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[16 * gl + 4 * i + e] = pack_bf16(__fmaf_rn(f[e], S, c), __fmaf_rn(f[4 + e], S, c));
         }
     }
 }
@@ -383,7 +419,8 @@ struct ScaleCursor {
             in = gi < groups;
             if (in) a = row + 2 * gi;
         }
-        if (FMT == kFmtW4G64) v = ldg_nc_u16(a);
+        if (FMT == kFmtW4SB32) v = 0u;                    // scales travel inside the records
+        else if (FMT == kFmtW4G64) v = ldg_nc_u16(a);
         else v = ldg_nc_u32(a);
         mask = in ? 0xffffffffu : 0u;
         if (valid && ++t >= u.t1) {
@@ -402,7 +439,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsign
 
 template <int FMT, int KS, int MAXI>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcArgs<MAXI> p) {
-    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : KS;        // code bytes per row and stage
+    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : 144;   // code bytes per row and stage
     constexpr int AS = KS == 128 ? 4 : 2;                    // A slots (KS / 2 columns each)
     constexpr uint32_t ACOLS = KS / 2;
     constexpr uint32_t QCOLS = ACOLS / 4;                    // columns one dequantizing thread writes per stage
@@ -539,8 +576,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         bool live = get_unit(p, 0, u);
         if (live) t = u.t0;
         // this thread's code chunks within a stage's codes tile
-        const uint32_t cp0 = code_pos<RB>(r, FMT == kFmtW4G64 && KS == 128 ? h : 2 * h);
-        const uint32_t cp1 = code_pos<RB>(r, 2 * h + 1);
+        const uint32_t cp0 = code_pos<RB>(r, FMT == kFmtW4SB32 ? 1 + 2 * h : FMT == kFmtW4G64 && KS == 128 ? h : 2 * h);
+        const uint32_t cp1 = code_pos<RB>(r, FMT == kFmtW4SB32 ? 2 + 2 * h : 2 * h + 1);
+        const uint32_t cph = code_pos<RB>(r, 0);               // superblock record header
         uint32_t g = 0;
         int slot = 0, wrap = 0;
         bool ok = true;
@@ -557,7 +595,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 if (warp == 3 && lane == 0) RQ_TC_MARK(5, g);
                 const uint8_t* cs = smem + (size_t)slot * p.stage_bytes + p.codes_off;
                 const uint32_t ta = tmem + tl + kTmemA0 + (uint32_t)a * ACOLS + (uint32_t)h * QCOLS;
-                if (FMT == kFmtW4G64 && KS == 256) {          // 64 weights: chunks 2h, 2h+1, one group
+                if (FMT == kFmtW4SB32) {                      // 64 weights: groups 2h, 2h+1 of the record
+                    const uint4 hd = *reinterpret_cast<const uint4*>(cs + cph);
+                    const uint4 c0 = *reinterpret_cast<const uint4*>(cs + cp0);
+                    const uint4 c1 = *reinterpret_cast<const uint4*>(cs + cp1);
+                    uint32_t o[32];
+                    dq_sb32(hd, c0, c1, h, o);
+                    tmem_st32(ta, o);
+                } else if (FMT == kFmtW4G64 && KS == 256) {   // 64 weights: chunks 2h, 2h+1, one group
                     const uint4 c0 = *reinterpret_cast<const uint4*>(cs + cp0);
                     const uint4 c1 = *reinterpret_cast<const uint4*>(cs + cp1);
                     const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -705,7 +750,7 @@ bool encode(EncodeTiled enc, CUtensorMap* m, CUtensorMapDataType dt, int rank, c
 
 template <int FMT, int KS, int MAXI>
 cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
-    constexpr uint32_t RB = FMT == kFmtW4G64 ? KS / 2 : KS;
+    constexpr uint32_t RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : 144;
     const EncodeTiled enc = encoder();
     if (!enc) return cudaErrorNotSupported;
     TcArgs<MAXI> p = {};
@@ -734,7 +779,8 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
         const uint64_t xd[3] = {64, (uint64_t)M, (uint64_t)(w.K / 64)}, xs[2] = {(uint64_t)w.K * 2, 128};
         const uint32_t xb[3] = {64, (uint32_t)xrows, (uint32_t)(KS / 64)};
         if (!encode(enc, &it.cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w.codes, cd, cs, cb,
-                    RB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+                    RB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : RB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                                    : CU_TENSOR_MAP_SWIZZLE_NONE) ||
             !encode(enc, &it.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.x, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         it.scales = static_cast<const uint8_t*>(w.scales);
@@ -808,6 +854,8 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
 // K allows; int8 rows are 128 bytes at 128-K stages already.
 template <int FMT>
 cudaError_t launch_chunk(const WgemmArgs* a, int count, cudaStream_t st) {
+    if (FMT == kFmtW4SB32)                                  // K % 256 == 0: one record per row and stage
+        return count == 1 ? launch_fmt_tc<FMT, 256, 1>(a, 1, st) : launch_fmt_tc<FMT, 256, kTcMaxItems>(a, count, st);
     if (FMT == kFmtW4G64) {
         bool wide = a[0].M <= 64;
         for (int i = 0; i < count; ++i) wide = wide && (a[i].K % 256 == 0);
@@ -829,10 +877,14 @@ cudaError_t launch_chunks(const WgemmArgs* a, int count, cudaStream_t st) {
 
 }  // namespace
 
-bool tc_supported(int fmt, int M) { return M >= kTcMinM && (fmt == kFmtW4G64 || fmt == kFmtW8G16); }
+bool tc_supported(int fmt, int M) {
+    return M >= kTcMinM && (fmt == kFmtW4G64 || fmt == kFmtW8G16 || fmt == kFmtW4SB32);
+}
 
 cudaError_t launch_tc(const WgemmArgs* a, int count, cudaStream_t st) {
-    return a[0].fmt == kFmtW4G64 ? launch_chunks<kFmtW4G64>(a, count, st) : launch_chunks<kFmtW8G16>(a, count, st);
+    if (a[0].fmt == kFmtW4G64) return launch_chunks<kFmtW4G64>(a, count, st);
+    if (a[0].fmt == kFmtW8G16) return launch_chunks<kFmtW8G16>(a, count, st);
+    return launch_chunks<kFmtW4SB32>(a, count, st);
 }
 
 cudaError_t status_tc(cudaStream_t st, unsigned* word) {

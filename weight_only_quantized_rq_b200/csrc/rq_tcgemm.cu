@@ -84,7 +84,7 @@ namespace {
 constexpr int kTcRows = 128;        // weight rows per tile (MMA M)
 constexpr int kTcMaxStages = 16;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemA0 = 256;   // first column of the A slots; D buffers below
+constexpr int kMaxAS = 8;           // A slots at most (the accumulators take the first columns)
 constexpr int kDqThreads = 512;     // warps 3-18
 constexpr int kEpiThreads = 128;    // warps 19-22
 constexpr int kTcThreads = 736;
@@ -110,6 +110,8 @@ struct TcArgs {
     TcItem it[MAXI];
     int count, units, M, Mpad, split, R;
     int niss;                       // MMA-issuing warps (two accumulators when Mpad <= 64)
+    int AS;                         // A slots in tensor memory
+    uint32_t A0;                    // first tensor-memory column of the A slots (after 2 * niss accumulators)
     uint32_t stage_bytes, x_atom, codes_off, bar_off, tx_bytes;
 };
 
@@ -431,16 +433,51 @@ struct ScaleCursor {
     }
 };
 
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity, sleeping about nap_ns between
+// tests. A blocking try_wait keeps its warp issuing while it polls, and with
+// 23 warps per CTA most of them wait most of the time: sleeping waiters leave
+// the issue slots to the warps that dequantize. Gives up after kWaitLimitNs,
+// ORs `flag` into the status word and returns false.
+__device__ __forceinline__ bool nap_wait(uint64_t* bar, uint32_t parity, unsigned flag, unsigned nap_ns) {
+    if (mbar_test(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(nap_ns);
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, flag);
+            return false;
+        }
+    }
+}
+
 // Bounded wait by every lane of a warp; true only if all lanes saw the phase.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned flag) {
-    const bool ok = mbar_wait_bounded(bar, parity, flag);
+// nap_ns == 0: waits on the critical path (dequantizing warps, MMA issue) use
+// the suspending try_wait, which measured faster there than sleeping between
+// tests; the long waits (epilogue, drains) sleep.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned flag, unsigned nap_ns) {
+    const bool ok = nap_ns ? nap_wait(bar, parity, flag, nap_ns) : mbar_wait_bounded(bar, parity, flag);
     return __all_sync(0xffffffffu, ok);
 }
+
+// Sleep between phase tests, by waiter (ns; 0 = suspending try_wait).
+constexpr unsigned kNapCritical = 0, kNapLoader = 64, kNapEpilogue = 512, kNapDrain = 256;
 
 template <int FMT, int KS, int MAXI>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcArgs<MAXI> p) {
     constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : 144;   // code bytes per row and stage
-    constexpr int AS = KS == 128 ? 4 : 2;                    // A slots (KS / 2 columns each)
+    const int AS = p.AS;                                     // A slots (KS / 2 columns each)
     constexpr uint32_t ACOLS = KS / 2;
     constexpr uint32_t QCOLS = ACOLS / 4;                    // columns one dequantizing thread writes per stage
     constexpr int NAT = KS / 64;                             // 64-K atoms per stage
@@ -453,8 +490,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
     uint64_t* empty = full + kTcMaxStages;
     uint64_t* afull = empty + kTcMaxStages;
-    uint64_t* aempty = afull + 4;
-    uint64_t* dfull = aempty + 4;
+    uint64_t* aempty = afull + kMaxAS;
+    uint64_t* dfull = aempty + kMaxAS;
     uint64_t* dempty = dfull + 2;
     uint64_t* mmadone = dempty + 2;                          // one per issuer
     uint32_t* tslot = reinterpret_cast<uint32_t*>(mmadone + 2);
@@ -499,26 +536,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             const uint32_t idesc = mma_idesc(Mpad);
             bool ok = true;
             uint32_t g = 0;
-            int slot = 0;
+            int slot = 0, aslot = 0, awrap = 0;
             Unit u;
             for (int ui = 0; ok && get_unit(p, ui, u); ++ui) {
                 const int d = ui & 1;
-                if (ui >= 2 && !warp_wait(&dempty[d], (uint32_t)((ui >> 1) - 1) & 1u, kStatusMmaWait)) {
+                if (ui >= 2 && !warp_wait(&dempty[d], (uint32_t)((ui >> 1) - 1) & 1u, kStatusMmaWait, kNapDrain)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t dcol = tmem + (uint32_t)((d * niss + w) * Mpad);
                 for (int t = u.t0; t < u.t1; ++t, ++g) {
-                    const int a = (int)(g % AS);
-                    if (!warp_wait(&afull[a], (g / AS) & 1u, kStatusTmaWait)) {
+                    const int a = aslot;
+                    if (!warp_wait(&afull[a], (uint32_t)awrap & 1u, kStatusTmaWait, kNapCritical)) {
                         ok = false;
                         break;
                     }
                     if (w == 0) RQ_TC_MARK(2, g);
                     tc_fence_after();
                     const uint32_t xs = base + (uint32_t)slot * p.stage_bytes;
-                    const uint32_t acol = tmem + kTmemA0 + (uint32_t)a * ACOLS;
+                    const uint32_t acol = tmem + p.A0 + (uint32_t)a * ACOLS;
                     const uint64_t bd = sw128_desc(xs);
                     const uint64_t xstep = (uint64_t)(p.x_atom >> 4);
                     for (int at = w; at < NAT; at += niss)
@@ -528,11 +565,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     mma_commit(&aempty[a]);
                     if (w == 0) RQ_TC_MARK(3, g);
                     if (++slot == R) slot = 0;
+                    if (++aslot == AS) { aslot = 0; ++awrap; }
                 }
                 if (ok) mma_commit(&dfull[d]);
             }
             mma_commit(&mmadone[w]);
-            warp_wait(&mmadone[w], 0u, kStatusMmaWait);      // no MMA in flight at teardown
+            warp_wait(&mmadone[w], 0u, kStatusMmaWait, kNapDrain);      // no MMA in flight at teardown
         }
     } else if (warp == 2) {
         // ------------------------------------------------------ tensor copies (one thread)
@@ -545,7 +583,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             for (int ui = 0; ok && get_unit(p, ui, u); ++ui) {
                 const TcItem& it = p.it[u.item];
                 for (int t = u.t0; t < u.t1; ++t, ++g) {
-                    if (wrap && !mbar_wait_bounded(&empty[slot], (uint32_t)(wrap - 1) & 1u, kStatusSlotWait, 64u)) {
+                    if (wrap && !nap_wait(&empty[slot], (uint32_t)(wrap - 1) & 1u, kStatusSlotWait, kNapLoader)) {
                         ok = false;
                         break;
                     }
@@ -580,7 +618,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         const uint32_t cp1 = code_pos<RB>(r, FMT == kFmtW4SB32 ? 2 + 2 * h : 2 * h + 1);
         const uint32_t cph = code_pos<RB>(r, 0);               // superblock record header
         uint32_t g = 0;
-        int slot = 0, wrap = 0;
+        int slot = 0, wrap = 0, aslot = 0, awrap = 0;
         bool ok = true;
         while (ok && live) {
 #pragma unroll
@@ -588,13 +626,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 if (!live) break;
                 const uint32_t s = sq[i] & sm[i];
                 sc.next(sq[i], sm[i]);
-                if (!warp_wait(&full[slot], (uint32_t)wrap & 1u, kStatusTmaWait)) { ok = false; break; }
+                if (!warp_wait(&full[slot], (uint32_t)wrap & 1u, kStatusTmaWait, kNapCritical)) { ok = false; break; }
                 if (warp == 3 && lane == 0) RQ_TC_MARK(4, g);
-                const int a = (int)(g % AS);
-                if (g >= AS && !warp_wait(&aempty[a], ((g / AS) - 1) & 1u, kStatusMmaWait)) { ok = false; break; }
+                const int a = aslot;
+                if (awrap && !warp_wait(&aempty[a], (uint32_t)(awrap - 1) & 1u, kStatusMmaWait, kNapCritical)) { ok = false; break; }
                 if (warp == 3 && lane == 0) RQ_TC_MARK(5, g);
                 const uint8_t* cs = smem + (size_t)slot * p.stage_bytes + p.codes_off;
-                const uint32_t ta = tmem + tl + kTmemA0 + (uint32_t)a * ACOLS + (uint32_t)h * QCOLS;
+                const uint32_t ta = tmem + tl + p.A0 + (uint32_t)a * ACOLS + (uint32_t)h * QCOLS;
                 if (FMT == kFmtW4SB32) {                      // 64 weights: groups 2h, 2h+1 of the record
                     const uint4 hd = *reinterpret_cast<const uint4*>(cs + cph);
                     const uint4 c0 = *reinterpret_cast<const uint4*>(cs + cp0);
@@ -628,6 +666,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 mbar_arrive(&afull[a]);
                 if (warp == 3 && lane == 0) RQ_TC_MARK(6, g);
                 if (++slot == R) { slot = 0; ++wrap; }
+                if (++aslot == AS) { aslot = 0; ++awrap; }
                 ++g;
                 if (++t >= u.t1) {
                     live = get_unit(p, ++ui, u);
@@ -645,7 +684,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         Unit u;
         for (int ui = 0; get_unit(p, ui, u); ++ui) {
             const int d = ui & 1;
-            if (!warp_wait(&dfull[d], (uint32_t)(ui >> 1) & 1u, kStatusMmaWait)) break;
+            if (!warp_wait(&dfull[d], (uint32_t)(ui >> 1) & 1u, kStatusMmaWait, kNapEpilogue)) break;
             if (warp == 19 && lane == 0) RQ_TC_MARK(7, ui);
             tc_fence_after();
             const TcItem& it = p.it[u.item];
@@ -794,6 +833,10 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
     }
     p.units = units;
     p.niss = p.Mpad <= 64 ? 2 : 1;
+    p.A0 = (uint32_t)(2 * p.niss * p.Mpad + 31) & ~31u;       // accumulator columns, then the A ring
+    p.AS = (int)((kTmemCols - p.A0) / (KS / 2));
+    if (p.AS > kMaxAS) p.AS = kMaxAS;
+    if (p.AS < 2) return cudaErrorInvalidValue;
     const int sms = sm_count();
     p.split = 1;
     if (count == 1 && units < sms / 2) {                     // too few tiles: split K over a cluster
@@ -810,7 +853,7 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
     const uint32_t codes_b = kTcRows * RB;
     p.stage_bytes = (p.codes_off + codes_b + 1023u) & ~1023u;
     p.tx_bytes = x_b + codes_b;                              // tensor-copy bytes per stage (boxes incl. zero fill)
-    const size_t bars = (2 * kTcMaxStages + 2 * 4 + 6) * 8 + 16;
+    const size_t bars = (2 * kTcMaxStages + 2 * kMaxAS + 6) * 8 + 16;
     const size_t avail = kTcSmemMax - 1024 - bars;
     int R = (int)(avail / p.stage_bytes);
     R = R > kTcMaxStages ? kTcMaxStages : R;

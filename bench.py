@@ -426,6 +426,23 @@ def run_ours(args, w, M):
             if w2 is not w:
                 del mats2
                 torch.cuda.empty_cache()
+    # the E[x^2] statistic of the scale search over a calibration batch of
+    # 7.2B width (32768 rows x 4096 channels of bf16, 256 MB > L2)
+    act_stats = None
+    if not args.quick:
+        R_c, K_c = 32768, 4096
+        g_c = torch.Generator(device=dev).manual_seed(77)
+        xa = torch.randn(R_c, K_c, device=dev, generator=g_c).to(torch.bfloat16)
+        ss = torch.zeros(K_c, dtype=torch.float64, device=dev)
+        f = capture(lambda: rq.rq_act_sumsq(xa, ss, stream=stream))
+        ms_a = timed(f, min(args.steps, 10))
+        gbs = R_c * K_c * 2 / (ms_a * 1e-3) / 1e9
+        act_stats = {"rows": R_c, "K": K_c, "ms_per_call": round(ms_a, 5), "GB_s": round(gbs, 2),
+                     "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": hbm, "unit": "GB/s",
+                                  "frac": round(gbs / hbm, 4),
+                                  "note": "algorithmic bytes = R * K * 2 (x read once) per call"},
+                     "kernel": "act_sumsq_kernel"}
+        del xa, ss
     status = rq.rq_device_status(stream)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
@@ -449,6 +466,7 @@ def run_ours(args, w, M):
         "configs_note": "per (configuration, M): one graph-captured step of batched launches over the "
                         "configuration's products; roofline_frac = sum over products of max(bytes / HBM peak, "
                         "flops / bf16 peak) divided by the step time",
+        "act_stats": act_stats,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": prob.h2d,
                 "d2h_bytes_per_step": prob.d2h},

@@ -16,7 +16,8 @@
  *          small-M GEMM / tensor-core GEMM family serves batches up to 32.
  *   [rwkv_quant_nv] "rwkv_quant_nv" project description, section "Operator
  *          Optimization Details": decode tile shapes for the 4096x4096,
- *          16384x4096 and 4096x16384 projections; r/k/v fused in one kernel.
+ *          16384x4096 and 4096x16384 projections; r/k/v fused in one kernel;
+ *          the activation statistic of its path computed on the device.
  *
  * Conventions shared by every call:
  *   - W is stored [N][K] row-major (row n = output feature, K = input
@@ -145,8 +146,9 @@ int rq_quantize_pack(const float *W, int K, int N, const float *act_sq,
  *   K,N must equal the descriptor's
  *   w   packed matrix
  *   y   device fp32 [M][N], overwritten (not accumulated into)
- * w_hat is formed in registers or shared memory and never written out; the
- * products accumulate in fp32. Kernels are launched with programmatic
+ * w_hat is formed in registers (M <= 2: CUDA-core GEMV, exact fp32 w_hat) or
+ * in tensor memory (M >= 3: tensor-core kernel, w_hat rounded once to bf16)
+ * and never written out; the products accumulate in fp32. Kernels are launched with programmatic
  * dependent launch allowed: they read the packed weights while the kernel
  * launched just before them on the stream may still be running, and read x
  * and write y only after it has completed. So the packed planes must not be
@@ -167,8 +169,10 @@ typedef struct rq_wgemm_item {
  * projections of a layer ([rwkv_quant_nv] "Operator Optimization Details":
  * r/k/v computed in a single kernel). Every item has the same format and the
  * same M; shapes may differ. The result equals `count` rq_wgemm calls. The
- * launch's CTAs split the items' packed bytes evenly, so small matrices
- * share the GPU instead of leaving it idle between launches.
+ * launch's CTAs split the items' work evenly (packed bytes for M <= 2,
+ * 128-row tiles for M >= 3), so small matrices share the GPU instead of
+ * leaving it idle between launches; above 96 items the tensor-core path
+ * takes one launch per 96 items.
  *   items  host array of `count` items, 1 <= count <= 160
  *   M      activation rows of every item, 1..128
  * No y may overlap another item's y or any x. Same validation, status codes
@@ -181,6 +185,28 @@ int rq_wgemm_batch(const rq_wgemm_item *items, int count, int M, void *stream);
  * same device unpack as rq_wgemm; bit-exact: q * scale for the symmetric
  * formats, fp32(S_j * q - M_j) for the superblock format. */
 int rq_dequant(const rq_packed *w, float *W_out, void *stream);
+
+/* Accumulate the statistic of the E[x^2]-weighted search on the device.
+ * ([ART] "Two presets and six sizes": the search weights input channel k by
+ * E[x_k^2]; [rwkv_quant_nv] "Operator Optimization Details": the activation
+ * statistic is computed on the device.)
+ *   x       device bf16 [R][K], calibration activations (raw bf16 bits)
+ *   sum_sq  device fp64 [K], caller-owned running sums: the call adds
+ *           sum_r x[r][k]^2 to sum_sq[k]. Zero it before the first batch;
+ *           call once per batch of rows.
+ * Summation order (deterministic, bit-reproducible): the R rows are cut into
+ * 64 contiguous chunks of ceil(R / 64) rows (the last ones may be short or
+ * empty); each chunk is summed in fp64 in ascending row order starting from
+ * 0, the 64 chunk sums are added in ascending chunk order starting from 0,
+ * and that total is added to sum_sq[k]. Squares of bf16 values are exact in
+ * fp64. Limits: 1 <= R <= 2^24, 1 <= K <= 2^20. Non-finite x: unspecified. */
+int rq_act_sumsq(const void *x, int R, int K, double *sum_sq, void *stream);
+
+/* act_sq[k] = fp32(sum_sq[k] / rows) (one fp64 division, one rounding to
+ * fp32), the E[x^2] that rq_quantize_pack takes.
+ *   sum_sq  device fp64 [K] from rq_act_sumsq; act_sq device fp32 [K];
+ *   rows    total calibration rows summed, >= 1. */
+int rq_act_finalize(const double *sum_sq, int K, long long rows, float *act_sq, void *stream);
 
 /* Static description of a status code. Never NULL. */
 const char *rq_status_string(int status);

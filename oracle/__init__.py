@@ -1,5 +1,6 @@
 """CPU oracle for weight-only group quantization (RTN and E[x^2]-weighted
-search), packing, exact dequantization and the fp64 product.
+search), packing, exact dequantization, the fp64 product and the activation
+statistic E[x^2].
 
 TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package. The product library
@@ -76,6 +77,10 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_dequant.restype = None
     L.orc_wgemm.argtypes = [_i, _P, _i, _i, _i, _P, _P, _P, _i, _P]
     L.orc_wgemm.restype = None
+    L.orc_act_sumsq.argtypes = [_P, _i, _i, _P]
+    L.orc_act_sumsq.restype = None
+    L.orc_act_finalize.argtypes = [_P, _i, ctypes.c_longlong, _P]
+    L.orc_act_finalize.restype = None
     L.orc_threads.argtypes = []
     L.orc_threads.restype = _i
     L.orc_set_threads.argtypes = [_i]
@@ -242,3 +247,23 @@ def wgemm(fmt: str, x_bf16_bits, K: int, N: int, codes, scales, rows=None) -> np
     y = np.zeros((M, nr), dtype=np.float64)
     lib().orc_wgemm(FORMATS[fmt], _ptr(x), M, K, N, _ptr(codes), _ptr(scales), _ptr(r), nr, _ptr(y))
     return y
+
+
+def act_sumsq(x_bf16_bits, sum_sq=None) -> np.ndarray:
+    """Running per-channel sums of x^2 over the rows of x (raw bf16 bits,
+    uint16 [R][K]) added into ``sum_sq`` (fp64 [K], zeros when None), in the
+    order of the design notes: 64 contiguous row chunks, each summed ascending,
+    then the chunk sums ascending."""
+    x = _c(x_bf16_bits, np.uint16)
+    R, K = x.shape
+    out = np.zeros(K, dtype=np.float64) if sum_sq is None else np.array(sum_sq, dtype=np.float64, copy=True)
+    lib().orc_act_sumsq(_ptr(x), R, K, _ptr(out))
+    return out
+
+
+def act_finalize(sum_sq, rows: int) -> np.ndarray:
+    """E[x^2] = fp32(sum_sq / rows)."""
+    s = _c(sum_sq, np.float64)
+    out = np.zeros(s.size, dtype=np.float32)
+    lib().orc_act_finalize(_ptr(s), s.size, int(rows), _ptr(out))
+    return out

@@ -462,6 +462,42 @@ void orc_wgemm(int fmt, const uint16_t *x, int M, int K, int N, const uint8_t *c
     free(xd);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Activation statistic E[x^2]                                              */
+/* ------------------------------------------------------------------------ */
+
+/* [ART] "Two presets and six sizes": the search weights input channel k by
+ * E[x_k^2], the mean over calibration rows of the squared activation. The
+ * pages fix no summation order; the reading here (the same for the device
+ * call) is: cut the R rows into 64 contiguous chunks of ceil(R / 64) rows,
+ * sum each chunk in fp64 in ascending row order starting from 0, add the 64
+ * chunk sums in ascending order starting from 0, and add that total to the
+ * running sum of channel k. x[r][k]^2 of a bf16 value is exact in fp64. */
+void orc_act_sumsq(const uint16_t *x, int R, int K, double *sum_sq)
+{
+    int rc = (R + 63) / 64;
+    for (int k = 0; k < K; k++) {
+        double total = 0.0;
+        for (int c = 0; c < 64; c++) {
+            int r0 = c * rc < R ? c * rc : R;
+            int r1 = r0 + rc < R ? r0 + rc : R;
+            double part = 0.0;
+            for (int r = r0; r < r1; r++) {
+                double v = (double)orc_bf16_to_f32(x[(size_t)r * K + k]);
+                part = part + v * v;
+            }
+            total = total + part;
+        }
+        sum_sq[k] = sum_sq[k] + total;
+    }
+}
+
+/* E[x_k^2] = fp32(sum_sq[k] / rows): one fp64 division, one rounding. */
+void orc_act_finalize(const double *sum_sq, int K, long long rows, float *act_sq)
+{
+    for (int k = 0; k < K; k++) act_sq[k] = (float)(sum_sq[k] / (double)rows);
+}
+
 /* Number of OpenMP threads a parallel region would use (0 without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

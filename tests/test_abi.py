@@ -152,3 +152,19 @@ def test_wgemm_batch_validation(L):
     nul = Items(rq.RqWgemmItem(0x40000, ctypes.pointer(d1), 0x50000),
                 rq.RqWgemmItem(0x60000, None, 0x70000))
     assert L.rq_wgemm_batch(nul, 2, 1, st) == rq.RQ_ERR_INVALID_ARG
+
+
+def test_act_stats_validation(L):
+    """The E[x^2] calls reject bad arguments on the host (nothing launched)."""
+    A, U, st = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8), None
+    assert L.rq_act_sumsq(None, 4, 64, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_sumsq(A, 4, 64, None, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_sumsq(A, 0, 64, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_sumsq(A, 4, 0, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_sumsq(A, (1 << 24) + 1, 64, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_sumsq(U, 4, 64, A, st) == rq.RQ_ERR_MISALIGNED
+    assert L.rq_act_sumsq(A, 4, 64, U, st) == rq.RQ_ERR_MISALIGNED
+    assert L.rq_act_finalize(None, 64, 4, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_finalize(A, 64, 0, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_finalize(A, 0, 4, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_act_finalize(A, 64, 4, U, st) == rq.RQ_ERR_MISALIGNED

@@ -35,6 +35,10 @@ MUTANTS = [
      "float s = orc_f16_to_f32(scales[(size_t)n * ng]);", None),
     ("sb dequant adds the min", "float p = (float)q * S;\n    return p - M;", "float p = (float)q * S;\n    return p + M;", None),
     ("absmax from the last element", "if (v > absmax) absmax = v;", "absmax = v;", None),
+    ("E[x^2] sums |x| instead of x^2", "part = part + v * v;", "part = part + fabs(v);", None),
+    ("E[x^2] skips the last chunk", "for (int c = 0; c < 64; c++) {\n            int r0", "for (int c = 0; c < 63; c++) {\n            int r0", None),
+    ("E[x^2] divides by rows - 1", "act_sq[k] = (float)(sum_sq[k] / (double)rows);", "act_sq[k] = (float)(sum_sq[k] / (double)(rows - 1));", None),
+    ("E[x^2] overwrites the running sum", "sum_sq[k] = sum_sq[k] + total;", "sum_sq[k] = total;", None),
 ]
 
 

@@ -453,3 +453,49 @@ def test_format_sizes_match_the_pages(orc):
     int4 = L * sum(packed_bytes(orc, "w4g64", k, n) for k, n in proj) + 2 * V * C * 2
     assert abs(fp16 / 1e9 - c["fp16_GB"]) <= c["rel_tol"] * c["fp16_GB"]
     assert abs(int4 / 1e9 - c["int4_GB"]) <= c["rel_tol"] * c["int4_GB"]
+
+
+# ----------------------------------------------------- E[x^2] statistic ---
+def _bf16_bits(a):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("R", [1, 3, 64, 65, 128, 1000])
+def test_act_stats_constant_rows(orc, R):
+    """Rows all equal to c (exact in bf16): E[x^2] = c^2 exactly."""
+    K = 5
+    c = np.array([1.5, -2.0, 0.0, 3.25, -0.125], np.float32)
+    x = np.tile(c, (R, 1))
+    got = orc.act_finalize(orc.act_sumsq(_bf16_bits(x)), R)
+    assert np.array_equal(got, (c.astype(np.float64) ** 2).astype(np.float32))
+
+
+def test_act_stats_integer_rows_exact(orc):
+    """Small-integer activations: every partial sum is an exact integer in
+    fp64, so the result is the integer sum of squares over R, rounded once."""
+    rng = np.random.default_rng(31)
+    R, K = 4097, 67           # 64 chunks of 65 rows: the last chunk holds 2 rows
+    xi = rng.integers(-40, 41, size=(R, K))
+    s = orc.act_sumsq(_bf16_bits(xi.astype(np.float32)))
+    assert np.array_equal(s, (xi.astype(np.int64) ** 2).sum(0).astype(np.float64))
+    assert np.array_equal(orc.act_finalize(s, R), ((xi.astype(np.int64) ** 2).sum(0) / R).astype(np.float32))
+
+
+def test_act_stats_match_numpy_and_accumulate(orc):
+    """Random bf16 activations with a massive channel: the fp64 sums agree
+    with numpy's to 1e-12, and two batches accumulate to the one-shot sum."""
+    rng = np.random.default_rng(32)
+    R, K = 1000, 96
+    x = rng.standard_normal((R, K)).astype(np.float32)
+    x[:, 7] *= 50.0
+    b = _bf16_bits(x)
+    xf = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = (xf ** 2).sum(0)
+    s = orc.act_sumsq(b)
+    assert np.allclose(s, ref, rtol=1e-12, atol=0)
+    s2 = orc.act_sumsq(b[600:], orc.act_sumsq(b[:600]))
+    assert np.allclose(s2, ref, rtol=1e-12, atol=0)
+    a = orc.act_finalize(s, R)
+    assert np.allclose(a, (ref / R).astype(np.float32), rtol=1e-6, atol=0)
+    assert int(np.argmax(a)) == 7

@@ -35,6 +35,7 @@ RQ_W8_SYM_G16 = 2
 RQ_W4_ASYM_SB32 = 3
 FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_ASYM_SB32}
 EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_dequant",
+           "rq_act_sumsq", "rq_act_finalize",
            "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
 MAX_BATCH = 160
 TC_MIN_M = 3         # activation rows from which int4 g64 / int8 g16 products run on the tensor cores
@@ -86,6 +87,10 @@ def _lib() -> ctypes.CDLL:
         L.rq_wgemm_batch.restype = I
         L.rq_dequant.argtypes = [ctypes.POINTER(RqPacked), P, P]
         L.rq_dequant.restype = I
+        L.rq_act_sumsq.argtypes = [P, I, I, P, P]
+        L.rq_act_sumsq.restype = I
+        L.rq_act_finalize.argtypes = [P, I, ctypes.c_longlong, P, P]
+        L.rq_act_finalize.restype = I
         L.rq_status_string.argtypes = [I]
         L.rq_status_string.restype = ctypes.c_char_p
         L.rq_last_cuda_error.argtypes = []
@@ -222,6 +227,27 @@ def rq_dequant(w: Packed, out: torch.Tensor | None = None, stream=None) -> torch
         out = torch.empty(w.N, w.K, dtype=torch.float32, device=w.codes.device)
     d = w.desc()
     _check(_lib().rq_dequant(ctypes.byref(d), _ptr(out), _stream(stream)), "rq_dequant")
+    return out
+
+
+def rq_act_sumsq(x: torch.Tensor, sum_sq: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Add sum_r x[r][k]^2 (x bf16 [R][K] on the GPU) into the fp64 running
+    sums sum_sq[K] (created as zeros when None) and return them."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 [R][K] tensor")
+    R, K = int(x.shape[0]), int(x.shape[1])
+    if sum_sq is None:
+        sum_sq = torch.zeros(K, dtype=torch.float64, device=x.device)
+    _check(_lib().rq_act_sumsq(_ptr(x), R, K, _ptr(sum_sq), _stream(stream)), "rq_act_sumsq")
+    return sum_sq
+
+
+def rq_act_finalize(sum_sq: torch.Tensor, rows: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """E[x^2] = fp32(sum_sq / rows), the act_sq that rq_quantize_pack takes."""
+    K = int(sum_sq.shape[0])
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=sum_sq.device)
+    _check(_lib().rq_act_finalize(_ptr(sum_sq), K, int(rows), _ptr(out), _stream(stream)), "rq_act_finalize")
     return out
 
 

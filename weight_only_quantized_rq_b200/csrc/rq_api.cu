@@ -132,6 +132,20 @@ int rq_dequant(const rq_packed* w, float* W_out, void* stream) {
                                           static_cast<cudaStream_t>(stream)));
 }
 
+int rq_act_sumsq(const void* x, int R, int K, double* sum_sq, void* stream) {
+    if (!x || !sum_sq) return RQ_ERR_INVALID_ARG;
+    if (R < 1 || R > (1 << 24) || K < 1 || K > (1 << 20)) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(sum_sq)) return RQ_ERR_MISALIGNED;
+    return cuda_status(rq::launch_act_sumsq(x, R, K, sum_sq, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_act_finalize(const double* sum_sq, int K, long long rows, float* act_sq, void* stream) {
+    if (!sum_sq || !act_sq) return RQ_ERR_INVALID_ARG;
+    if (K < 1 || K > (1 << 20) || rows < 1) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(sum_sq) || !aligned16(act_sq)) return RQ_ERR_MISALIGNED;
+    return cuda_status(rq::launch_act_finalize(sum_sq, K, rows, act_sq, static_cast<cudaStream_t>(stream)));
+}
+
 const char* rq_status_string(int status) {
     switch (status) {
         case RQ_OK: return "ok";

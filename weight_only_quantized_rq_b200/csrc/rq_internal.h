@@ -58,6 +58,11 @@ constexpr int kTcMinM = 3;
 bool tc_supported(int fmt, int M);
 cudaError_t launch_tc(const WgemmArgs* a, int count, cudaStream_t st);
 
+// Per-channel sums of squares of bf16 activations (adds into sum_sq) and
+// their finalization into fp32 E[x^2].
+cudaError_t launch_act_sumsq(const void* x, int R, int K, double* sum_sq, cudaStream_t st);
+cudaError_t launch_act_finalize(const double* sum_sq, int K, long long rows, float* act_sq, cudaStream_t st);
+
 // Read and clear the device status word of each kernel file (synchronizes st).
 cudaError_t status_pack(cudaStream_t st, unsigned* word);
 cudaError_t status_gemv(cudaStream_t st, unsigned* word);

@@ -9,8 +9,8 @@ CPU-baseline leg of ``bench.py`` may import this package. The product library
 The arithmetic lives in ``rq_oracle.c`` (plain C loops, IEEE fp32/fp64, no
 contraction, no fast-math); this module only compiles it and marshals numpy
 arrays. Formats are named by strings here: ``"w4g64"`` (symmetric int4, group
-64), ``"w8g16"`` (symmetric int8, group 16), ``"w4sb32"`` (asymmetric int4
-superblock of 8 groups of 32).
+64), ``"w8g16"`` (symmetric int8, group 16), ``"w4sb32"`` / ``"w5sb32"`` /
+``"w6sb32"`` (asymmetric 4-, 5-, 6-bit superblocks of 8 groups of 32).
 """
 from __future__ import annotations
 
@@ -25,8 +25,10 @@ _SRC = os.path.join(_HERE, "rq_oracle.c")
 _OUT_DIR = os.path.join(_HERE, "_build")
 _SO = os.path.join(_OUT_DIR, "librq_oracle.so")
 
-FORMATS = {"w4g64": 1, "w8g16": 2, "w4sb32": 3}
-GROUP = {"w4g64": 64, "w8g16": 16, "w4sb32": 32}
+FORMATS = {"w4g64": 1, "w8g16": 2, "w4sb32": 3, "w5sb32": 4, "w6sb32": 5}
+GROUP = {"w4g64": 64, "w8g16": 16, "w4sb32": 32, "w5sb32": 32, "w6sb32": 32}
+SB_BITS = {"w4sb32": 4, "w5sb32": 5, "w6sb32": 6}
+SB_BYTES = {"w4sb32": 144, "w5sb32": 176, "w6sb32": 208}
 QMAX = {"w4g64": 7, "w8g16": 127}
 
 _P = ctypes.c_void_p
@@ -63,15 +65,15 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_grid.restype = None
     L.orc_sym_group.argtypes = [_P, _P, _i, _i, _P, _i, _P, _P, _P]
     L.orc_sym_group.restype = _i
-    L.orc_asym_group.argtypes = [_P, _P, _i, _P, _i, _P, _P, _P]
+    L.orc_asym_group.argtypes = [_P, _P, _i, _P, _i, _i, _P, _P, _P]
     L.orc_asym_group.restype = _i
-    L.orc_sb_finish.argtypes = [_P, _P, _P, _P]
+    L.orc_sb_finish.argtypes = [_P, _P, _P, _i, _P]
     L.orc_sb_finish.restype = None
     L.orc_sb_field.argtypes = [_P, _i, _i]
     L.orc_sb_field.restype = _i
     L.orc_pack_sym.argtypes = [_P, _i, _i, _P, _i, _i, _f, _f, _P, _P]
     L.orc_pack_sym.restype = None
-    L.orc_pack_sb32.argtypes = [_P, _i, _i, _P, _i, _f, _f, _P]
+    L.orc_pack_sb32.argtypes = [_P, _i, _i, _P, _i, _f, _f, _i, _P]
     L.orc_pack_sb32.restype = None
     L.orc_dequant.argtypes = [_i, _i, _i, _P, _P, _P]
     L.orc_dequant.restype = None
@@ -171,25 +173,26 @@ def sym_group(w, a, qmax: int, n: int = 64, t_lo: float = 0.7, t_hi: float = 1.0
     return idx, int(s[0]), q, losses
 
 
-def asym_group(w, a, n: int = 64, t_lo: float = 0.7, t_hi: float = 1.0):
-    """Search one asymmetric group. Returns (index, S*, M*, losses)."""
+def asym_group(w, a, n: int = 64, t_lo: float = 0.7, t_hi: float = 1.0, bits: int = 4):
+    """Search one asymmetric group of `bits`-bit codes. Returns (index, S*, M*, losses)."""
     w = _c(w, np.float32)
     a = None if a is None else _c(a, np.float32)
     t = grid(n, t_lo, t_hi)
     S = np.zeros(1, dtype=np.float32)
     M = np.zeros(1, dtype=np.float32)
     losses = np.zeros(n, dtype=np.float64)
-    idx = lib().orc_asym_group(_ptr(w), _ptr(a), w.size, _ptr(t), n, _ptr(S), _ptr(M), _ptr(losses))
+    idx = lib().orc_asym_group(_ptr(w), _ptr(a), w.size, _ptr(t), n, bits, _ptr(S), _ptr(M), _ptr(losses))
     return idx, float(S[0]), float(M[0]), losses
 
 
-def sb_finish(w256, S_star, M_star) -> np.ndarray:
-    """The 144-byte superblock record for 256 weights and 8 searched (S*, M*)."""
+def sb_finish(w256, S_star, M_star, bits: int = 4) -> np.ndarray:
+    """The superblock record (144 / 176 / 208 bytes for 4 / 5 / 6 bits) for
+    256 weights and 8 searched (S*, M*)."""
     w = _c(w256, np.float32)
     S = _c(S_star, np.float32)
     M = _c(M_star, np.float32)
-    blk = np.zeros(144, dtype=np.uint8)
-    lib().orc_sb_finish(_ptr(w), _ptr(S), _ptr(M), _ptr(blk))
+    blk = np.zeros(16 + 128 + (bits - 4) * 32, dtype=np.uint8)
+    lib().orc_sb_finish(_ptr(w), _ptr(S), _ptr(M), bits, _ptr(blk))
     return blk
 
 
@@ -205,8 +208,8 @@ def packed_shapes(fmt: str, K: int, N: int):
         return (N, K // 2), np.uint8, (N, K // 64)
     if fmt == "w8g16":
         return (N, K), np.uint8, (N, K // 16)
-    if fmt == "w4sb32":
-        return (N, (K // 256) * 144), np.uint8, None
+    if fmt in SB_BYTES:
+        return (N, (K // 256) * SB_BYTES[fmt]), np.uint8, None
     raise ValueError(fmt)
 
 
@@ -217,8 +220,8 @@ def pack(fmt: str, W, act_sq=None, n_cand: int = 64, t_lo: float = 0.7, t_hi: fl
     a = None if act_sq is None else _c(act_sq, np.float32)
     cshape, cdt, sshape = packed_shapes(fmt, K, N)
     codes = np.zeros(cshape, dtype=cdt)
-    if fmt == "w4sb32":
-        lib().orc_pack_sb32(_ptr(W), K, N, _ptr(a), n_cand, t_lo, t_hi, _ptr(codes))
+    if fmt in SB_BITS:
+        lib().orc_pack_sb32(_ptr(W), K, N, _ptr(a), n_cand, t_lo, t_hi, SB_BITS[fmt], _ptr(codes))
         return codes, None
     scales = np.zeros(sshape, dtype=np.uint16)
     lib().orc_pack_sym(_ptr(W), K, N, _ptr(a), FORMATS[fmt], n_cand, t_lo, t_hi,

@@ -48,6 +48,13 @@
 #define ORC_W4G64 1
 #define ORC_W8G16 2
 #define ORC_W4SB32 3
+#define ORC_W5SB32 4
+#define ORC_W6SB32 5
+
+/* Bits per code and record bytes of the superblock formats (4, 5, 6 bits:
+ * 144, 176, 208 bytes per 256 weights). */
+static int sb_bits(int fmt) { return fmt == ORC_W6SB32 ? 6 : (fmt == ORC_W5SB32 ? 5 : 4); }
+static int sb_bytes(int bits) { return 16 + 128 + (bits - 4) * 32; }
 
 /* ------------------------------------------------------------------------ */
 /* Number formats                                                           */
@@ -247,12 +254,12 @@ void orc_pack_sym(const float *W, int K, int N, const float *a, int fmt,
 /* ------------------------------------------------------------------------ */
 
 /* Codes of one asymmetric group with scale S and min offset M (w_hat = S*q - M):
- *   q = clamp(rint((w + M) / S), 0, 15),  and q = 0 when S == 0. */
-static int asym_code(float w, float S, float M)
+ *   q = clamp(rint((w + M) / S), 0, L),  L = 2^bits - 1,  and q = 0 when S == 0. */
+static int asym_code(float w, float S, float M, int L)
 {
     if (S == 0.0f) return 0;
     float v = (w + M) / S;
-    return (int)rintf(clampf(v, 0.0f, 15.0f));
+    return (int)rintf(clampf(v, 0.0f, (float)L));
 }
 
 static float asym_deq(int q, float S, float M)
@@ -261,19 +268,22 @@ static float asym_deq(int q, float S, float M)
     return p - M;
 }
 
-/* One asymmetric group of G (= 32) weights: the E[x^2]-weighted scale/shift
- * search of [ART] applied to the COMPRESSION preset's asymmetric layout.
+/* One asymmetric group of G (= 32) weights with codes of `bits` bits: the
+ * E[x^2]-weighted scale/shift search of [ART] applied to the COMPRESSION
+ * preset's asymmetric layout (4 bits for projections; 5 and 6 bits for the
+ * channel-mix key, head, embedding and LoRA weights of that preset).
  * The pages name the search but not its candidates; the reading taken here:
- *   lo = min(0, min w), hi = max(0, max w)
+ *   lo = min(0, min w), hi = max(0, max w), levels = 2^bits - 1
  *   candidate i shrinks [lo, hi] about its midpoint by t_i:
  *     half = (hi - lo) * 0.5,  mid = (hi + lo) * 0.5,  r = t_i * half
- *     S_i = (2r) / 15,  M_i = max(0, -(mid - r))
+ *     S_i = (2r) / levels,  M_i = max(0, -(mid - r))
  *   w_hat = S_i * q - M_i (fp32 multiply, then fp32 subtract), loss as in the
  *   symmetric case, lowest index on ties.
  * Returns the chosen index; writes the fp32 (S*, M*) of the winner. */
-int orc_asym_group(const float *w, const float *a, int G, const float *t, int n,
+int orc_asym_group(const float *w, const float *a, int G, const float *t, int n, int bits,
                    float *S_out, float *M_out, double *losses)
 {
+    const int levels = (1 << bits) - 1;
     float lo = 0.0f, hi = 0.0f;
     for (int k = 0; k < G; k++) {
         if (w[k] < lo) lo = w[k];
@@ -286,12 +296,12 @@ int orc_asym_group(const float *w, const float *a, int G, const float *t, int n,
     float bS = 0.0f, bM = 0.0f;
     for (int i = 0; i < n; i++) {
         float r = t[i] * half;
-        float S = (2.0f * r) / 15.0f;
+        float S = (2.0f * r) / (float)levels;
         float lo_i = mid - r;
         float M = (lo_i < 0.0f) ? -lo_i : 0.0f;
         double L = 0.0;
         for (int k = 0; k < G; k++) {
-            float wq = asym_deq(asym_code(w[k], S, M), S, M);
+            float wq = asym_deq(asym_code(w[k], S, M, levels), S, M);
             double d = (double)w[k] - (double)wq;
             double e = d * d;
             double ak = a ? (double)a[k] : 1.0;
@@ -305,21 +315,28 @@ int orc_asym_group(const float *w, const float *a, int G, const float *t, int n,
     return best;
 }
 
-/* Finish one superblock of 8 groups x 32 weights into its 144-byte record.
- * The layout is this project's own (the pages give only "asymmetric
- * superblock, group 32"; the 6-bit scale/min against an fp16 superblock
- * scale/min is the stated configuration):
+/* Finish one superblock of 8 groups x 32 weights into its record (144, 176
+ * or 208 bytes for 4-, 5- or 6-bit codes). The layout is this project's own
+ * (the pages give only "asymmetric superblock, group 32"; the 6-bit
+ * scale/min against an fp16 superblock scale/min is the stated
+ * configuration; 5 and 6 bits add exactly 1 and 2 bits per weight, the
+ * file-size deltas [ART] quotes for o_proj):
  *   [0:2]    fp16 d      = fp16(max_j S*_j / 63)
  *   [2:4]    fp16 dmin   = fp16(max_j M*_j / 63)
  *   [4:16]   96-bit little-endian bit string: bits 6j..6j+5 hold sc_j,
  *            bits 48+6j..48+6j+5 hold m_j (j = 0..7)
  *            sc_j = clamp(rint(S*_j / d), 0, 63), 0 when d == 0; m_j likewise
- *   [16:144] 128 code bytes, low nibble k = 2t, high nibble k = 2t+1, code = q
+ *   [16:144] 128 bytes of the codes' low 4 bits: low nibble k = 2t, high
+ *            nibble k = 2t+1
+ *   5 bits:  [144:176] bit 4 of code k in bit k % 8 of byte 144 + k / 8
+ *   6 bits:  [144:208] bits 4..5 of code k in bits 2 (k % 4) .. +1 of byte
+ *            144 + k / 4
  * The final codes use the stored values S_j = d * sc_j and M_j = dmin * m_j
  * (both exact fp32 products); there is no second search after the 6-bit
  * rounding. */
-void orc_sb_finish(const float *w, const float *S_star, const float *M_star, uint8_t *blk)
+void orc_sb_finish(const float *w, const float *S_star, const float *M_star, int bits, uint8_t *blk)
 {
+    const int levels = (1 << bits) - 1;
     float mS = 0.0f, mM = 0.0f;
     for (int j = 0; j < 8; j++) {
         if (S_star[j] > mS) mS = S_star[j];
@@ -333,7 +350,7 @@ void orc_sb_finish(const float *w, const float *S_star, const float *M_star, uin
         sc[j] = (d == 0.0f) ? 0 : (int)rintf(clampf(S_star[j] / d, 0.0f, 63.0f));
         mc[j] = (dm == 0.0f) ? 0 : (int)rintf(clampf(M_star[j] / dm, 0.0f, 63.0f));
     }
-    memset(blk, 0, 144);
+    memset(blk, 0, (size_t)sb_bytes(bits));
     blk[0] = (uint8_t)(dh & 0xff); blk[1] = (uint8_t)(dh >> 8);
     blk[2] = (uint8_t)(mh & 0xff); blk[3] = (uint8_t)(mh >> 8);
     for (int j = 0; j < 8; j++) {
@@ -348,18 +365,23 @@ void orc_sb_finish(const float *w, const float *S_star, const float *M_star, uin
         float M = dm * (float)mc[j];
         for (int k = 0; k < 32; k++) {
             int kk = 32 * j + k;
-            int q = asym_code(w[kk], S, M);
-            if ((kk & 1) == 0) blk[16 + kk / 2] = (uint8_t)q;
-            else blk[16 + kk / 2] |= (uint8_t)(q << 4);
+            int q = asym_code(w[kk], S, M, levels);
+            int lo4 = q & 15, up = q >> 4;
+            if ((kk & 1) == 0) blk[16 + kk / 2] = (uint8_t)lo4;
+            else blk[16 + kk / 2] |= (uint8_t)(lo4 << 4);
+            if (bits == 5) blk[144 + kk / 8] |= (uint8_t)(up << (kk % 8));
+            if (bits == 6) blk[144 + kk / 4] |= (uint8_t)(up << (2 * (kk % 4)));
         }
     }
 }
 
-/* Pack a whole [N][K] matrix (K % 256 == 0) into [N][K/256] superblocks. */
+/* Pack a whole [N][K] matrix (K % 256 == 0) into [N][K/256] superblocks of
+ * `bits`-bit codes. */
 void orc_pack_sb32(const float *W, int K, int N, const float *a, int n_cand,
-                   float t_lo, float t_hi, uint8_t *blocks)
+                   float t_lo, float t_hi, int bits, uint8_t *blocks)
 {
     int nb = K / 256;
+    size_t rs = (size_t)sb_bytes(bits);
     float *t = (float *)malloc(sizeof(float) * (size_t)n_cand);
     orc_grid(n_cand, t_lo, t_hi, t);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -369,9 +391,9 @@ void orc_pack_sb32(const float *W, int K, int N, const float *a, int n_cand,
             float S[8], M[8];
             for (int j = 0; j < 8; j++) {
                 size_t k0 = (size_t)b * 256 + (size_t)j * 32;
-                orc_asym_group(row + k0, a ? a + k0 : NULL, 32, t, n_cand, &S[j], &M[j], NULL);
+                orc_asym_group(row + k0, a ? a + k0 : NULL, 32, t, n_cand, bits, &S[j], &M[j], NULL);
             }
-            orc_sb_finish(row + (size_t)b * 256, S, M, blocks + ((size_t)n * nb + b) * 144);
+            orc_sb_finish(row + (size_t)b * 256, S, M, bits, blocks + ((size_t)n * nb + b) * rs);
         }
     }
     free(t);
@@ -399,10 +421,11 @@ int orc_sb_field(const uint8_t *blk, int which, int j)
 static void deq_row(int fmt, int K, const uint8_t *codes, const uint16_t *scales,
                     int n, float *out)
 {
-    if (fmt == ORC_W4SB32) {
-        int nb = K / 256;
+    if (fmt == ORC_W4SB32 || fmt == ORC_W5SB32 || fmt == ORC_W6SB32) {
+        int nb = K / 256, bits = sb_bits(fmt);
+        size_t rs = (size_t)sb_bytes(bits);
         for (int b = 0; b < nb; b++) {
-            const uint8_t *blk = codes + ((size_t)n * nb + b) * 144;
+            const uint8_t *blk = codes + ((size_t)n * nb + b) * rs;
             float d = orc_f16_to_f32((uint16_t)(blk[0] | (blk[1] << 8)));
             float dm = orc_f16_to_f32((uint16_t)(blk[2] | (blk[3] << 8)));
             for (int j = 0; j < 8; j++) {
@@ -411,6 +434,8 @@ static void deq_row(int fmt, int K, const uint8_t *codes, const uint16_t *scales
                 for (int k = 0; k < 32; k++) {
                     int kk = 32 * j + k;
                     int q = (blk[16 + kk / 2] >> (4 * (kk & 1))) & 0xf;
+                    if (bits == 5) q |= ((blk[144 + kk / 8] >> (kk % 8)) & 1) << 4;
+                    if (bits == 6) q |= ((blk[144 + kk / 4] >> (2 * (kk % 4))) & 3) << 4;
                     out[(size_t)b * 256 + kk] = asym_deq(q, S, M);
                 }
             }

@@ -23,7 +23,9 @@ MUTANTS = [
     ("truncate instead of rint", "float r = rintf(clampf(v, -(float)qmax, (float)qmax));",
      "float r = truncf(clampf(v, -(float)qmax, (float)qmax));", None),
     ("asym offset sign", "float M = (lo_i < 0.0f) ? -lo_i : 0.0f;", "float M = (lo_i < 0.0f) ? lo_i : 0.0f;", None),
-    ("asym step over 16 levels", "float S = (2.0f * r) / 15.0f;", "float S = (2.0f * r) / 16.0f;", None),
+    ("asym step over 2^b levels", "float S = (2.0f * r) / (float)levels;", "float S = (2.0f * r) / (float)(levels + 1);", None),
+    ("5-bit plane bit order", "blk[144 + kk / 8] |= (uint8_t)(up << (kk % 8));", "blk[144 + kk / 8] |= (uint8_t)(up << (7 - kk % 8));", None),
+    ("6-bit plane uses 1 bit per code", "blk[144 + kk / 4] |= (uint8_t)(up << (2 * (kk % 4)));", "blk[144 + kk / 4] |= (uint8_t)((up & 1) << (2 * (kk % 4)));", None),
     ("bit string off by one", "int bs = 6 * j + b, bm = 48 + 6 * j + b;", "int bs = 6 * j + b, bm = 47 + 6 * j + b;", None),
     ("fp16 ties away from zero", "(rem == halfway && (kept & 1u))", "(rem == halfway)", None),
     ("grid misses its top end", "step = step / (double)(n - 1);", "step = step / (double)n;", None),

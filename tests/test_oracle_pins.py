@@ -304,6 +304,44 @@ def test_exact_products_sb32(orc):
     assert np.array_equal(y, want.astype(np.float64))
 
 
+@pytest.mark.parametrize("fmt,bits", [("w5sb32", 5), ("w6sb32", 6)])
+def test_exact_products_sb_wide(orc, fmt, bits):
+    """5- and 6-bit superblocks: w = S_j (q - 2^(bits-1)) with S_j = c_j 2^-12
+    (c_j <= 63, one group per superblock at 63) and codes spanning
+    0..2^bits - 1: the t = 1 candidate is exact, d = 2^-12, dmin =
+    2^(bits-13), sc_j = m_j = c_j, and weights and product come back exactly."""
+    rng = np.random.default_rng(42 + bits)
+    L, h = (1 << bits) - 1, 1 << (bits - 1)
+    N, K, M = 5, 512, 2
+    q = rng.integers(0, L + 1, size=(N, K))
+    qg = q.reshape(N, K // 32, 32)
+    qg[:, :, 0] = 0
+    qg[:, :, 1] = L
+    c = rng.integers(1, 64, size=(N, K // 32))
+    c.reshape(N, -1, 8)[:, :, 5] = 63
+    S = c.repeat(32, axis=1).astype(np.float64) * 2.0 ** -12
+    W = (S * (q - h)).astype(np.float32)
+    assert np.array_equal(W.astype(np.float64), S * (q - h))
+    codes, _ = orc.pack(fmt, W, None, n_cand=64)
+    blk = codes.reshape(N, K // 256, orc.SB_BYTES[fmt])
+    assert np.all(blk[..., 0:2].copy().view(np.uint16) == np.float16(2.0 ** -12).view(np.uint16))
+    assert np.all(blk[..., 2:4].copy().view(np.uint16) == np.float16(2.0 ** (bits - 13)).view(np.uint16))
+    assert np.array_equal(orc.dequant(fmt, K, N, codes, None), W)
+    # the stored codes decode to q: low nibbles plus the high-bit plane
+    lo = np.stack([blk[..., 16:144] & 15, blk[..., 16:144] >> 4], -1).reshape(N, K // 256, 256)
+    plane = blk[..., 144:]
+    if bits == 5:
+        up = np.unpackbits(plane, axis=-1, bitorder="little").reshape(N, K // 256, 256)
+    else:
+        up = np.stack([(plane >> (2 * i)) & 3 for i in range(4)], -1).reshape(N, K // 256, 256)
+    assert np.array_equal((lo | (up << 4)).reshape(N, K), q)
+    xi = rng.integers(-8, 9, size=(M, K))
+    xb = (xi.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    y = orc.wgemm(fmt, xb, K, N, codes, None)
+    want = (xi[:, None, :] * (c.repeat(32, axis=1) * (q - h))[None]).sum(-1) * 2.0 ** -12
+    assert np.array_equal(y, want.astype(np.float64))
+
+
 # ---------------------------------------- superblock fields, brute force ---
 def test_sb_fields_and_codes_brute_force(orc):
     rng = np.random.default_rng(51)
@@ -346,7 +384,7 @@ def test_sb_fields_and_codes_brute_force(orc):
                 assert qk == max(0, min(15, nearest_int_even(v)))
 
 
-def brute_asym(w, a, t):
+def brute_asym(w, a, t, levels=15):
     """Exact-rational loss of every candidate of the asymmetric reading
     (shrink [min(0,min w), max(0,max w)] about its midpoint by t_i; the step
     S = 2r/15 and offset M = max(0, r - mid) formed with numpy fp32 ops),
@@ -358,7 +396,7 @@ def brute_asym(w, a, t):
     out = []
     for ti in t:
         r = np.float32(np.float32(ti) * half)
-        S = np.float32(np.float32(2.0) * r / np.float32(15.0))
+        S = np.float32(np.float32(2.0) * r / np.float32(levels))
         loi = np.float32(mid - r)
         M = np.float32(-loi) if loi < 0 else np.float32(0.0)
         L = Fr(0)
@@ -366,15 +404,16 @@ def brute_asym(w, a, t):
             if S == 0:
                 q = 0
             else:
-                q = max(0, min(15, nearest_int_even((Fr(float(wk)) + Fr(float(M))) / Fr(float(S)))))
+                q = max(0, min(levels, nearest_int_even((Fr(float(wk)) + Fr(float(M))) / Fr(float(S)))))
             wh = Fr(float(np.float32(np.float32(q) * S) - M))
             L += Fr(float(ak)) * (Fr(float(wk)) - wh) ** 2
         out.append((L, float(S), float(M)))
     return out
 
 
+@pytest.mark.parametrize("bits", [4, 5, 6])
 @pytest.mark.parametrize("seed", range(6))
-def test_asym_search_matches_exact_brute_force(orc, seed):
+def test_asym_search_matches_exact_brute_force(orc, seed, bits):
     rng = np.random.default_rng(100 + seed)
     w = (rng.standard_normal(32) * 0.02).astype(np.float32)
     if seed == 1:
@@ -385,26 +424,28 @@ def test_asym_search_matches_exact_brute_force(orc, seed):
     if seed % 2:
         a[rng.integers(32)] = 15631.0
     t = orc.grid(64)
-    idx, S, M, _ = orc.asym_group(w, a, 64)
-    bl = brute_asym(w, a, t)
+    idx, S, M, _ = orc.asym_group(w, a, 64, bits=bits)
+    bl = brute_asym(w, a, t, (1 << bits) - 1)
     bidx = min(range(64), key=lambda i: (bl[i][0], i))
     if idx != bidx:
         assert abs(bl[idx][0] - bl[bidx][0]) <= Fr(1, 10**12) * bl[bidx][0]
     assert (S, M) == (bl[idx][1], bl[idx][2])
 
 
-def test_asym_t1_covers_the_group_range(orc):
-    """With the single candidate t = 1 the representable range [-M, 15S - M]
-    covers [min(0, min w), max(0, max w)] and every weight is within S/2 (plus
-    fp32 rounding) of its dequantized value."""
+@pytest.mark.parametrize("bits", [4, 5, 6])
+def test_asym_t1_covers_the_group_range(orc, bits):
+    """With the single candidate t = 1 the representable range [-M, L S - M]
+    (L = 2^bits - 1) covers [min(0, min w), max(0, max w)] and every weight is
+    within S/2 (plus fp32 rounding) of its dequantized value."""
     rng = np.random.default_rng(61)
+    L = (1 << bits) - 1
     for rep in range(50):
         w = (rng.standard_normal(32) * 0.02 * (1 + rep)).astype(np.float32)
-        _, S, M, _ = orc.asym_group(w, None, 1)
+        _, S, M, _ = orc.asym_group(w, None, 1, bits=bits)
         lo, hi = min(0.0, float(w.min())), max(0.0, float(w.max()))
-        assert -M <= lo * (1 - 1e-6) + 1e-12 and 15 * S - M >= hi * (1 - 1e-6) - 1e-12
+        assert -M <= lo * (1 - 1e-6) + 1e-12 and L * S - M >= hi * (1 - 1e-6) - 1e-12
         for wk in w:
-            q = max(0, min(15, round((float(wk) + M) / S)))
+            q = max(0, min(L, round((float(wk) + M) / S)))
             assert abs(float(wk) - (S * q - M)) <= S / 2 * (1 + 1e-5)
 
 
@@ -442,6 +483,12 @@ def test_format_sizes_match_the_pages(orc):
     per_bit = c["layers"] * c["K"] * c["N"] / 8
     assert round(per_bit / 1e6, 1) == c["plus_1bit_MB"]
     assert round(2 * per_bit / 1e6, 1) == c["plus_2bit_MB"]
+    # the 5- and 6-bit superblock records carry exactly those deltas
+    base = packed_bytes(orc, "w4sb32", c["K"], c["N"])
+    d5 = c["layers"] * (packed_bytes(orc, "w5sb32", c["K"], c["N"]) - base)
+    d6 = c["layers"] * (packed_bytes(orc, "w6sb32", c["K"], c["N"]) - base)
+    assert round(d5 / 1e6, c["decimals"]) == c["plus_1bit_MB"]
+    assert round(d6 / 1e6, c["decimals"]) == c["plus_2bit_MB"]
     c = g["w4sb32_first_o_proj_range"]
     for C in c["widths"]:
         d = C * C * 2 - packed_bytes(orc, "w4sb32", C, C)

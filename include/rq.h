@@ -77,11 +77,24 @@ typedef enum rq_status {
  *     [16:144] 128 code bytes, nibble order as RQ_W4_SYM_G64, code = q in [0, 15]
  *   Group j: S_j = d * sc_j, M_j = dmin * m_j; w_hat = S_j * q - M_j
  *   (S_j * q exact, one fp32 rounding). 4.5 bits per weight; scales = NULL.
+ *
+ * RQ_W5_ASYM_SB32, RQ_W6_ASYM_SB32 ([ART], the COMPRESSION preset's wider
+ *   matrices; +1 and +2 bits per weight, the o_proj file-size deltas the
+ *   article quotes): the RQ_W4_ASYM_SB32 record with the codes' low 4 bits in
+ *   [16:144] and a high-bit plane appended; q in [0, 31] or [0, 63]:
+ *     5 bits, 176-byte records: [144:176] bit 4 of code k in bit k % 8 of
+ *             byte 144 + k / 8
+ *     6 bits, 208-byte records: [144:208] bits 4..5 of code k in bits
+ *             2 (k % 4) .. 2 (k % 4) + 1 of byte 144 + k / 4
+ *   The group search spans 2^b - 1 steps (S = 2 r / (2^b - 1)); the rest is
+ *   as RQ_W4_ASYM_SB32. 5.5 and 6.5 bits per weight; scales = NULL.
  */
 typedef enum rq_format {
     RQ_W4_SYM_G64 = 1,
     RQ_W8_SYM_G16 = 2,
-    RQ_W4_ASYM_SB32 = 3
+    RQ_W4_ASYM_SB32 = 3,
+    RQ_W5_ASYM_SB32 = 4,
+    RQ_W6_ASYM_SB32 = 5
 } rq_format;
 
 /* Candidate grid of the E[x^2]-weighted search ([ART]): n_cand points
@@ -96,8 +109,8 @@ typedef struct rq_search {
 } rq_search;
 
 /* Descriptor of one packed matrix. A host struct holding device pointers;
- * the caller fills it and owns both planes. scales is NULL for
- * RQ_W4_ASYM_SB32. */
+ * the caller fills it and owns both planes. scales is NULL for the
+ * superblock formats (RQ_W4/W5/W6_ASYM_SB32). */
 typedef struct rq_packed {
     int fmt;        /* rq_format */
     int K;          /* input features */
@@ -108,7 +121,7 @@ typedef struct rq_packed {
 } rq_packed;
 
 /* Shape limits: 1 <= N <= 2^24; 64 <= K <= 32768 with K % 64 == 0
- * (K % 256 == 0 for RQ_W4_ASYM_SB32); 1 <= M <= 128. */
+ * (K % 256 == 0 for the superblock formats); 1 <= M <= 128. */
 
 /* Bytes of the two planes of a packed [N][K] matrix; the scales plane is
  * rounded up to a multiple of 16 bytes (the padding is written as zero by
@@ -129,8 +142,9 @@ size_t rq_packed_size(int fmt, int K, int N, size_t *codes_bytes, size_t *scales
  * evaluated in fp64 in ascending k; the lowest index attaining the minimum
  * wins. For each asymmetric group of 32: lo = min(0, min w),
  * hi = max(0, max w), candidate i shrinks [lo, hi] about its midpoint by t_i
- * (S_i = 2 r_i / 15, M_i = max(0, r_i - mid), r_i = t_i (hi - lo) / 2),
- * codes q = clamp(rint((w + M_i) / S_i), 0, 15), the same loss and tie rule;
+ * (S_i = 2 r_i / L, M_i = max(0, r_i - mid), r_i = t_i (hi - lo) / 2,
+ * L = 2^b - 1 = 15, 31 or 63 for b-bit codes),
+ * codes q = clamp(rint((w + M_i) / S_i), 0, L), the same loss and tie rule;
  * then d = fp16(max_j S_j / 63), dmin = fp16(max_j M_j / 63), 6-bit
  * sc_j = rint(S_j / d), m_j = rint(M_j / dmin), and the final codes use the
  * stored S_j = d sc_j, M_j = dmin m_j. The output is byte-for-byte
@@ -147,7 +161,8 @@ int rq_quantize_pack(const float *W, int K, int N, const float *act_sq,
  *   w   packed matrix
  *   y   device fp32 [M][N], overwritten (not accumulated into)
  * w_hat is formed in registers (M <= 2: CUDA-core GEMV, exact fp32 w_hat) or
- * in tensor memory (M >= 3: tensor-core kernel, w_hat rounded once to bf16)
+ * in tensor memory (M >= 3, and every M for the 5- and 6-bit formats:
+ * tensor-core kernel, w_hat rounded once to bf16)
  * and never written out; the products accumulate in fp32. Kernels are launched with programmatic
  * dependent launch allowed: they read the packed weights while the kernel
  * launched just before them on the stream may still be running, and read x
@@ -183,7 +198,7 @@ int rq_wgemm_batch(const rq_wgemm_item *items, int count, int M, void *stream);
 /* Export w_hat as fp32 [N][K] into W_out (device).  ([CARD] summary: the
  * kernel output is bit-identical to the offline dequantization.) Uses the
  * same device unpack as rq_wgemm; bit-exact: q * scale for the symmetric
- * formats, fp32(S_j * q - M_j) for the superblock format. */
+ * formats, fp32(S_j * q - M_j) for the superblock formats. */
 int rq_dequant(const rq_packed *w, float *W_out, void *stream);
 
 /* Accumulate the statistic of the E[x^2]-weighted search on the device.

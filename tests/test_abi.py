@@ -45,6 +45,8 @@ def test_version_and_status_strings(L):
     ("w4g64", 2048, 2048, 2048 * 1024, 2048 * 32 * 2),
     ("w8g16", 2048, 2048, 2048 * 2048, 2048 * 128 * 2),
     ("w4sb32", 2560, 2560, 2560 * 10 * 144, 0),
+    ("w5sb32", 2560, 2560, 2560 * 10 * 176, 0),
+    ("w6sb32", 256, 3, 3 * 208, 0),
     ("w4g64", 768, 3, 3 * 384, 80),        # 3 rows x 12 scales x 2 B = 72, padded to 80
 ])
 def test_packed_size(L, fmt, K, N, codes, scales):
@@ -57,13 +59,14 @@ def test_packed_size(L, fmt, K, N, codes, scales):
 
 def test_bits_per_weight(L):
     K = N = 4096
-    for fmt, bpw in [("w4g64", 4.25), ("w8g16", 9.0), ("w4sb32", 4.5)]:
+    for fmt, bpw in [("w4g64", 4.25), ("w8g16", 9.0), ("w4sb32", 4.5), ("w5sb32", 5.5), ("w6sb32", 6.5)]:
         cb, sb = rq.rq_packed_size(fmt, K, N)
         assert (cb + sb) * 8 / (K * N) == bpw
 
 
 @pytest.mark.parametrize("fmt,K,N", [("w4g64", 96, 4), ("w4sb32", 320, 4), ("w8g16", 65536, 4),
-                                     ("w4g64", 2048, 0), ("w4g64", 32, 1), (7, 2048, 2)])
+                                     ("w5sb32", 320, 4), ("w6sb32", 64, 4), ("w4g64", 2048, 0),
+                                     ("w4g64", 32, 1), (7, 2048, 2), (6, 2048, 2), (0, 2048, 2)])
 def test_packed_size_rejects(L, fmt, K, N):
     f = rq.fmt_id(fmt)
     assert L.rq_packed_size(f, K, N, None, None) == 0
@@ -91,8 +94,9 @@ def test_wgemm_validation(L):
     assert L.rq_wgemm(A, 1, 2048, 256, ctypes.byref(bad), A, st) == rq.RQ_ERR_MISALIGNED
     nos = _desc("w4g64", 2048, 256, scales=0)
     assert L.rq_wgemm(A, 1, 2048, 256, ctypes.byref(nos), A, st) == rq.RQ_ERR_INVALID_ARG
-    sb = _desc("w4sb32", 2048, 256)   # superblock format carries no scales plane
-    assert L.rq_wgemm(A, 1, 2048, 256, ctypes.byref(sb), A, st) == rq.RQ_ERR_FORMAT_MISMATCH
+    for f in ("w4sb32", "w5sb32", "w6sb32"):   # superblock formats carry no scales plane
+        sb = _desc(f, 2048, 256)
+        assert L.rq_wgemm(A, 1, 2048, 256, ctypes.byref(sb), A, st) == rq.RQ_ERR_FORMAT_MISMATCH
     res = _desc("w4g64", 2048, 256, reserved=1)
     assert L.rq_wgemm(A, 1, 2048, 256, ctypes.byref(res), A, st) == rq.RQ_ERR_FORMAT_MISMATCH
     odd = _desc("w4g64", 2080, 256)
@@ -119,8 +123,9 @@ def test_dequant_validation(L):
     assert L.rq_dequant(ctypes.byref(d), None, st) == rq.RQ_ERR_INVALID_ARG
     assert L.rq_dequant(ctypes.byref(d), U, st) == rq.RQ_ERR_MISALIGNED
     assert L.rq_dequant(None, A, st) == rq.RQ_ERR_INVALID_ARG
-    bad = _desc("w4sb32", 320, 8, scales=0)
-    assert L.rq_dequant(ctypes.byref(bad), A, st) == rq.RQ_ERR_UNSUPPORTED_SHAPE
+    for f in ("w4sb32", "w5sb32", "w6sb32"):
+        bad = _desc(f, 320, 8, scales=0)
+        assert L.rq_dequant(ctypes.byref(bad), A, st) == rq.RQ_ERR_UNSUPPORTED_SHAPE
 
 
 def test_binding_raises_without_library(monkeypatch, tmp_path):

@@ -73,12 +73,13 @@ def test_guard_band_and_padding():
     assert bool((big[:32] == 7.0).all()) and bool((big[32 + K:] == 7.0).all())
 
 
-@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w4sb32"])
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w4sb32", "w5sb32", "w6sb32"])
 def test_calibrate_then_pack_matches_oracle_chain(fmt):
     """Device statistic -> device pack gives the codes of oracle statistic ->
     oracle pack: the whole calibration path stays on the GPU."""
-    K, N, R = 2560 if fmt == "w4sb32" else 2048, 48, 512
-    x = calib(11, R, K, massive=517 if fmt == "w4sb32" else 1202)
+    sb = fmt.endswith("sb32")
+    K, N, R = 2560 if sb else 2048, 48, 512
+    x = calib(11, R, K, massive=517 if sb else 1202)
     W = wl.random_matrix(12, N, K)
     a_dev = rq.rq_act_finalize(rq.rq_act_sumsq(x.cuda()), R)
     p = rq.rq_quantize_pack(W.cuda(), fmt, a_dev, 64)

@@ -13,14 +13,14 @@ namespace {
 
 thread_local int t_last_cuda = 0;
 
-bool fmt_ok(int fmt) { return fmt == rq::kFmtW4G64 || fmt == rq::kFmtW8G16 || fmt == rq::kFmtW4SB32; }
+bool fmt_ok(int fmt) { return fmt == rq::kFmtW4G64 || fmt == rq::kFmtW8G16 || rq::is_sb(fmt); }
 
 // RQ_OK, or the status for an unsupported (fmt, K, N).
 int shape_status(int fmt, int K, int N) {
     if (!fmt_ok(fmt)) return RQ_ERR_INVALID_ARG;
     if (N < 1 || N > (1 << 24) || K < 64 || K > 32768) return RQ_ERR_INVALID_ARG;
     if (K % 64 != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
-    if (fmt == rq::kFmtW4SB32 && K % 256 != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+    if (rq::is_sb(fmt) && K % 256 != 0) return RQ_ERR_UNSUPPORTED_SHAPE;
     return RQ_OK;
 }
 
@@ -32,7 +32,7 @@ int check_packed(const rq_packed* w, int K, int N) {
     if (s != RQ_OK) return s;
     if (w->K != K || w->N != N || w->reserved != 0) return RQ_ERR_FORMAT_MISMATCH;
     if (!w->codes) return RQ_ERR_INVALID_ARG;
-    if (w->fmt == rq::kFmtW4SB32) {
+    if (rq::is_sb(w->fmt)) {
         if (w->scales) return RQ_ERR_FORMAT_MISMATCH;
     } else if (!w->scales) {
         return RQ_ERR_INVALID_ARG;
@@ -150,7 +150,7 @@ const char* rq_status_string(int status) {
     switch (status) {
         case RQ_OK: return "ok";
         case RQ_ERR_INVALID_ARG: return "invalid argument (NULL pointer, or M/K/N/search out of range)";
-        case RQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (K must be a multiple of 64; of 256 for the superblock format)";
+        case RQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (K must be a multiple of 64; of 256 for the superblock formats)";
         case RQ_ERR_FORMAT_MISMATCH: return "packed descriptor does not match the call (format, K or N)";
         case RQ_ERR_MISALIGNED: return "a device pointer is not 16-byte aligned";
         case RQ_ERR_CUDA: return "CUDA runtime error (see rq_last_cuda_error)";

@@ -898,7 +898,8 @@ cudaError_t launch_gemv(const WgemmArgs* a, int count, cudaStream_t st) {
     switch (a[0].fmt) {
         case kFmtW4G64: return launch_fmt<kFmtW4G64>(a, count, st);
         case kFmtW8G16: return launch_fmt<kFmtW8G16>(a, count, st);
-        default: return launch_fmt<kFmtW4SB32>(a, count, st);
+        case kFmtW4SB32: return launch_fmt<kFmtW4SB32>(a, count, st);
+        default: return cudaErrorNotSupported;            // 5- and 6-bit records run on the tensor-core kernel
     }
 }
 

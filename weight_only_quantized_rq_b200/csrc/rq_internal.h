@@ -11,11 +11,19 @@ namespace rq {
 constexpr int kFmtW4G64 = 1;
 constexpr int kFmtW8G16 = 2;
 constexpr int kFmtW4SB32 = 3;
+constexpr int kFmtW5SB32 = 4;
+constexpr int kFmtW6SB32 = 5;
 
-// Bytes per row of the codes plane (records plane for the superblock format)
+// The asymmetric superblock formats: bits per code and bytes per record of
+// 256 weights (16-byte header, 128 bytes of low nibbles, high-bit plane).
+__host__ __device__ constexpr bool is_sb(int fmt) { return fmt >= kFmtW4SB32 && fmt <= kFmtW6SB32; }
+__host__ __device__ constexpr int sb_bits(int fmt) { return fmt - kFmtW4SB32 + 4; }
+__host__ __device__ constexpr int sb_record(int fmt) { return 16 + 128 + (sb_bits(fmt) - 4) * 32; }
+
+// Bytes per row of the codes plane (records plane for the superblock formats)
 // and of the scales plane.
 inline size_t code_row_bytes(int fmt, int K) {
-    return fmt == kFmtW4G64 ? (size_t)K / 2 : fmt == kFmtW8G16 ? (size_t)K : (size_t)K / 256 * 144;
+    return fmt == kFmtW4G64 ? (size_t)K / 2 : fmt == kFmtW8G16 ? (size_t)K : (size_t)K / 256 * sb_record(fmt);
 }
 inline size_t scale_row_bytes(int fmt, int K) {
     return fmt == kFmtW4G64 ? (size_t)K / 32 : fmt == kFmtW8G16 ? (size_t)K / 8 : 0;

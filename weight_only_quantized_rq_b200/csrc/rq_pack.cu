@@ -41,10 +41,10 @@ __device__ __forceinline__ int sym_code(float w, float sf, float qmax) {
     return (int)rintf(clampf(__fdiv_rn(w, sf), -qmax, qmax));
 }
 
-// Asymmetric code: clamp(rint((w + M) / S), 0, 15); 0 if S == 0.
-__device__ __forceinline__ int asym_code(float w, float S, float M) {
+// Asymmetric code: clamp(rint((w + M) / S), 0, L), L = 2^bits - 1; 0 if S == 0.
+__device__ __forceinline__ int asym_code(float w, float S, float M, float L) {
     if (S == 0.0f) return 0;
-    return (int)rintf(clampf(__fdiv_rn(__fadd_rn(w, M), S), 0.0f, 15.0f));
+    return (int)rintf(clampf(__fdiv_rn(__fadd_rn(w, M), S), 0.0f, L));
 }
 
 // (loss, index) pair reduction over a warp: smallest loss, then smallest index.
@@ -125,16 +125,21 @@ qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restr
     if (lane == 0) scales[(size_t)n * ng + g] = __half_as_ushort(best_s);
 }
 
-// One block per superblock of 256 weights: warp j searches group j (32
-// weights), then the block forms d, dmin, the 6-bit fields and the codes.
+// One block per superblock of 256 weights with BITS-bit codes (4, 5, 6):
+// warp j searches group j (32 weights), then the block forms d, dmin, the
+// 6-bit fields, the codes' low nibbles and (5, 6 bits) the high-bit plane.
+template <int BITS>
 __global__ void __launch_bounds__(256)
-qpack_sb32_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
-                  int n_cand, float t_lo, float t_hi, uint8_t* __restrict__ blocks) {
+qpack_sb_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
+                int n_cand, float t_lo, float t_hi, uint8_t* __restrict__ blocks) {
+    constexpr int RS = 16 + 128 + (BITS - 4) * 32;          // record bytes
+    constexpr float kTop = (float)((1 << BITS) - 1);        // highest code
     __shared__ float s_w[256];
     __shared__ float s_a[256];
     __shared__ float s_S[8], s_M[8];     // searched S*_j, M*_j
     __shared__ float s_Sq[8], s_Mq[8];   // stored S_j = d sc_j, M_j = dmin m_j
-    __shared__ __align__(16) uint8_t s_blk[144];
+    __shared__ uint8_t s_q[256];         // final codes
+    __shared__ __align__(16) uint8_t s_blk[RS];
     const int nb = K / 256;
     const long long sb = blockIdx.x;
     const int n = (int)(sb / nb), b = (int)(sb % nb);
@@ -162,25 +167,25 @@ qpack_sb32_kernel(const float* __restrict__ W, int K, int N, const float* __rest
         int bestI = 0x7fffffff;
         for (int i = lane; i < n_cand; i += 32) {
             const float r = __fmul_rn(cand_t(i, n_cand, t_lo, t_hi), half);
-            const float S = __fdiv_rn(__fmul_rn(2.0f, r), 15.0f);
+            const float S = __fdiv_rn(__fmul_rn(2.0f, r), kTop);
             const float loi = __fsub_rn(mid, r);
             const float M = loi < 0.0f ? -loi : 0.0f;
-            double L = 0.0;
+            double loss = 0.0;
             if (n_cand > 1) {
                 for (int k = 0; k < 32; ++k) {
                     const float wk = w[k];
-                    const float wq = __fsub_rn(__fmul_rn((float)asym_code(wk, S, M), S), M);
+                    const float wq = __fsub_rn(__fmul_rn((float)asym_code(wk, S, M, kTop), S), M);
                     const double d = __dsub_rn((double)wk, (double)wq);
-                    L = __dadd_rn(L, __dmul_rn((double)a[k], __dmul_rn(d, d)));
+                    loss = __dadd_rn(loss, __dmul_rn((double)a[k], __dmul_rn(d, d)));
                 }
             }
-            if (bestI == 0x7fffffff || L < bestL) { bestL = L; bestI = i; }
+            if (bestI == 0x7fffffff || loss < bestL) { bestL = loss; bestI = i; }
         }
         warp_argmin(bestL, bestI);
         if (lane == 0) {
             const float r = __fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), half);
             const float loi = __fsub_rn(mid, r);
-            s_S[warp] = __fdiv_rn(__fmul_rn(2.0f, r), 15.0f);
+            s_S[warp] = __fdiv_rn(__fmul_rn(2.0f, r), kTop);
             s_M[warp] = loi < 0.0f ? -loi : 0.0f;
         }
     }
@@ -225,16 +230,26 @@ qpack_sb32_kernel(const float* __restrict__ W, int K, int N, const float* __rest
         }
     }
     __syncthreads();
-    if (t < 128) {   // code byte t: k = 2t (low nibble), 2t+1 (high)
-        const int j = (2 * t) >> 5;
-        const float S = s_Sq[j], M = s_Mq[j];
-        const int q0 = asym_code(s_w[2 * t], S, M);
-        const int q1 = asym_code(s_w[2 * t + 1], S, M);
-        s_blk[16 + t] = (uint8_t)(q0 | (q1 << 4));
+    s_q[t] = (uint8_t)asym_code(s_w[t], s_Sq[t >> 5], s_Mq[t >> 5], kTop);   // code of weight t
+    __syncthreads();
+    if (t < 128) {   // low-nibble byte t: k = 2t (low nibble), 2t+1 (high)
+        s_blk[16 + t] = (uint8_t)((s_q[2 * t] & 15) | ((s_q[2 * t + 1] & 15) << 4));
+    } else if (BITS == 5 && t < 160) {   // plane byte i: bit 4 of codes 8i .. 8i+7
+        const int i = t - 128;
+        uint32_t v = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v |= (uint32_t)((s_q[8 * i + e] >> 4) & 1) << e;
+        s_blk[144 + i] = (uint8_t)v;
+    } else if (BITS == 6 && t < 192) {   // plane byte i: bits 4..5 of codes 4i .. 4i+3
+        const int i = t - 128;
+        uint32_t v = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v |= (uint32_t)((s_q[4 * i + e] >> 4) & 3) << (2 * e);
+        s_blk[144 + i] = (uint8_t)v;
     }
     __syncthreads();
-    if (t < 9) {
-        uint4* dst = reinterpret_cast<uint4*>(blocks + ((size_t)n * nb + b) * 144);
+    if (t < RS / 16) {
+        uint4* dst = reinterpret_cast<uint4*>(blocks + ((size_t)n * nb + b) * RS);
         dst[t] = reinterpret_cast<const uint4*>(s_blk)[t];
     }
 }
@@ -282,9 +297,13 @@ __global__ void dequant_w8_kernel(const uint32_t* __restrict__ codes, const __ha
         make_float4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
 }
 
-// One thread per 32-bit word of a superblock's codes (32 words per record).
-__global__ void dequant_sb32_kernel(const uint8_t* __restrict__ blocks, int K, long long words,
-                                    float* __restrict__ out) {
+// One thread per 32-bit word of a superblock's low nibbles (32 words, 8
+// weights each, per record); the high-bit plane adds bits 4 (5-bit codes)
+// or 4..5 (6-bit codes).
+template <int BITS>
+__global__ void dequant_sb_kernel(const uint8_t* __restrict__ blocks, int K, long long words,
+                                  float* __restrict__ out) {
+    constexpr int RS = 16 + 128 + (BITS - 4) * 32;
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= words) return;
     const long long rec = i / 32;
@@ -292,7 +311,8 @@ __global__ void dequant_sb32_kernel(const uint8_t* __restrict__ blocks, int K, l
     const int nb = K / 256;
     const long long n = rec / nb;
     const int b = (int)(rec % nb);
-    const uint32_t* r = reinterpret_cast<const uint32_t*>(blocks + rec * 144);
+    const uint8_t* rb = blocks + rec * RS;
+    const uint32_t* r = reinterpret_cast<const uint32_t*>(rb);
     const uint32_t h0 = r[0];
     const float d = __half2float(__ushort_as_half((unsigned short)(h0 & 0xffffu)));
     const float dm = __half2float(__ushort_as_half((unsigned short)(h0 >> 16)));
@@ -301,8 +321,14 @@ __global__ void dequant_sb32_kernel(const uint8_t* __restrict__ blocks, int K, l
     const float M = __fmul_rn(dm, (float)sb_field(r[1], r[2], r[3], 1, j));
     float o[8];
     w4_word_values(r[4 + wi], o);
+    const uint32_t hb = BITS == 5 ? (uint32_t)rb[144 + wi]
+                      : BITS == 6 ? (uint32_t)rb[144 + 2 * wi] | ((uint32_t)rb[145 + 2 * wi] << 8) : 0u;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) o[s] = __fmaf_rn(S, __fsub_rn(o[s], 128.0f), -M);
+    for (int s = 0; s < 8; ++s) {
+        const float up = BITS == 5 ? (float)((hb >> s) & 1u) : BITS == 6 ? (float)((hb >> (2 * s)) & 3u) : 0.0f;
+        const float q = __fadd_rn(__fsub_rn(o[s], 128.0f), __fmul_rn(16.0f, up));   // exact small integer
+        o[s] = __fmaf_rn(S, q, -M);
+    }
     float4* dst = reinterpret_cast<float4*>(out + n * K + (size_t)b * 256 + wi * 8);
     dst[0] = make_float4(o[0], o[1], o[2], o[3]);
     dst[1] = make_float4(o[4], o[5], o[6], o[7]);
@@ -312,10 +338,12 @@ __global__ void dequant_sb32_kernel(const uint8_t* __restrict__ blocks, int K, l
 
 cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st) {
     const long long N = a.N;
-    if (a.fmt == kFmtW4SB32) {
+    if (is_sb(a.fmt)) {
         const long long blocksN = N * (a.K / 256);
-        qpack_sb32_kernel<<<(unsigned)blocksN, 256, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo, a.t_hi,
-                                                              static_cast<uint8_t*>(a.codes));
+        auto kern = a.fmt == kFmtW4SB32 ? qpack_sb_kernel<4> : a.fmt == kFmtW5SB32 ? qpack_sb_kernel<5>
+                                                                                : qpack_sb_kernel<6>;
+        kern<<<(unsigned)blocksN, 256, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo, a.t_hi,
+                                                static_cast<uint8_t*>(a.codes));
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         pack_done_kernel<<<1, 32, 0, st>>>();
@@ -357,8 +385,10 @@ cudaError_t launch_dequant(int fmt, int K, int N, const void* codes, const void*
             static_cast<const uint32_t*>(codes), static_cast<const __half*>(scales), K, words, out);
     } else {
         const long long words = (long long)N * (K / 256) * 32;
-        dequant_sb32_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
-            static_cast<const uint8_t*>(codes), K, words, out);
+        auto kern = fmt == kFmtW4SB32 ? dequant_sb_kernel<4> : fmt == kFmtW5SB32 ? dequant_sb_kernel<5>
+                                                                              : dequant_sb_kernel<6>;
+        kern<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(static_cast<const uint8_t*>(codes), K,
+                                                                             words, out);
     }
     return cudaGetLastError();
 }

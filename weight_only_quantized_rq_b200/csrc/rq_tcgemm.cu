@@ -346,6 +346,72 @@ __device__ __forceinline__ void dq_sb32(const uint4 hd, const uint4 c0, const ui
     }
 }
 
+// 5- and 6-bit superblock codes: the high-bit plane of one 32-bit word of low
+// nibbles (eight weights k = 0..7) becomes two words whose byte m holds the
+// high bits of weight 2m (hl) or 2m + 1 (hh) at bit 4 and up, so that OR-ing
+// them into the unpacked nibbles gives bytes 0..63 that the fp32 magic turns
+// into 128 + q exactly.
+// 5 bits: pw is the plane byte, bit k for weight k. The multiply moves bit 2m
+// to bit 8m + 4; the other partial products land elsewhere (and collide only
+// at bits 10, 16, 22, whose carries stop at 11, 17, 23), so the mask keeps
+// exactly the wanted bits.
+// 6 bits: pw holds 16 plane bits, bits 2k..2k+1 for weight k. After masking,
+// nibble m of e holds the pair of weight 2m; the byte permute places nibble m
+// in the high half of byte m (the low halves are masked off where used).
+template <int BITS>
+__device__ __forceinline__ void sb_high(uint32_t pw, uint32_t& hl, uint32_t& hh) {
+    if (BITS == 5) {
+        hl = ((pw & 0x55u) * 0x00410410u) & 0x10101010u;
+        hh = (((pw >> 1) & 0x55u) * 0x00410410u) & 0x10101010u;
+    } else {
+        const uint32_t e = pw & 0x3333u, o = (pw >> 2) & 0x3333u;
+        hl = prmt(e << 4, e, 0x5140u);
+        hh = prmt(o << 4, o, 0x5140u);
+    }
+}
+
+// (a & 0x0F0F0F0F) | (b & 0xF0F0F0F0)
+__device__ __forceinline__ uint32_t merge_nib(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(0x0F0F0F0Fu));
+    return d;
+}
+
+// 64 weights of a 5- or 6-bit record (groups 2h, 2h + 1): as dq_sb32, with
+// the high bits of each code from the plane words pl (two per group for 6
+// bits: words 2gl, 2gl + 1 of pl; one byte per code word for 5 bits).
+template <int BITS>
+__device__ __forceinline__ void dq_sbw(const uint4 hd, const uint4 c0, const uint4 c1, const uint32_t (&pl)[4], int h,
+                                       uint32_t (&o)[32]) {
+    const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
+    const float dmin = __half2float(__ushort_as_half((uint16_t)(hd.x >> 16)));
+#pragma unroll
+    for (int gl = 0; gl < 2; ++gl) {
+        const int j = 2 * h + gl;
+        const float S = __fmul_rn(d, (float)sb_field(hd.y, hd.z, hd.w, 0, j));
+        const float Mv = __fmul_rn(dmin, (float)sb_field(hd.y, hd.z, hd.w, 1, j));
+        const float c = __fsub_rn(__fmul_rn(-128.0f, S), Mv);
+        const uint4 cw = gl == 0 ? c0 : c1;
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t pw = BITS == 5 ? (pl[gl] >> (8 * i)) & 0xffu : (pl[2 * gl + (i >> 1)] >> (16 * (i & 1))) & 0xffffu;
+            uint32_t hl, hh;
+            sb_high<BITS>(pw, hl, hh);
+            const uint32_t lo = merge_nib(w[i], hl), hi = merge_nib(w[i] >> 4, hh);
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                f[e] = __uint_as_float(prmt(lo, kW4Magic, 0x7044u + 0x100u * e));
+                f[4 + e] = __uint_as_float(prmt(hi, kW4Magic, 0x7044u + 0x100u * e));
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[16 * gl + 4 * i + e] = pack_bf16(__fmaf_rn(f[e], S, c), __fmaf_rn(f[4 + e], S, c));
+        }
+    }
+}
+
 // ------------------------------------------------------------ work units
 struct Unit { int item, n0, t0, t1; };
 
@@ -421,7 +487,7 @@ struct ScaleCursor {
             in = gi < groups;
             if (in) a = row + 2 * gi;
         }
-        if (FMT == kFmtW4SB32) v = 0u;                    // scales travel inside the records
+        if (is_sb(FMT)) v = 0u;                           // scales travel inside the records
         else if (FMT == kFmtW4G64) v = ldg_nc_u16(a);
         else v = ldg_nc_u32(a);
         mask = in ? 0xffffffffu : 0u;
@@ -476,7 +542,7 @@ constexpr unsigned kNapCritical = 0, kNapLoader = 64, kNapEpilogue = 512, kNapDr
 
 template <int FMT, int KS, int MAXI>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcArgs<MAXI> p) {
-    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : 144;   // code bytes per row and stage
+    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : sb_record(FMT);   // code bytes per row and stage
     const int AS = p.AS;                                     // A slots (KS / 2 columns each)
     constexpr uint32_t ACOLS = KS / 2;
     constexpr uint32_t QCOLS = ACOLS / 4;                    // columns one dequantizing thread writes per stage
@@ -614,9 +680,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         bool live = get_unit(p, 0, u);
         if (live) t = u.t0;
         // this thread's code chunks within a stage's codes tile
-        const uint32_t cp0 = code_pos<RB>(r, FMT == kFmtW4SB32 ? 1 + 2 * h : FMT == kFmtW4G64 && KS == 128 ? h : 2 * h);
-        const uint32_t cp1 = code_pos<RB>(r, FMT == kFmtW4SB32 ? 2 + 2 * h : 2 * h + 1);
+        const uint32_t cp0 = code_pos<RB>(r, is_sb(FMT) ? 1 + 2 * h : FMT == kFmtW4G64 && KS == 128 ? h : 2 * h);
+        const uint32_t cp1 = code_pos<RB>(r, is_sb(FMT) ? 2 + 2 * h : 2 * h + 1);
         const uint32_t cph = code_pos<RB>(r, 0);               // superblock record header
+        // high-bit plane of groups 2h, 2h + 1: 8 bytes (5 bits) or 16 (6 bits) at 144 + 8h or 144 + 16h
+        const uint32_t cpp = code_pos<RB>(r, 0) + 144u + (FMT == kFmtW6SB32 ? 16u : 8u) * (uint32_t)h;
         uint32_t g = 0;
         int slot = 0, wrap = 0, aslot = 0, awrap = 0;
         bool ok = true;
@@ -639,6 +707,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     const uint4 c1 = *reinterpret_cast<const uint4*>(cs + cp1);
                     uint32_t o[32];
                     dq_sb32(hd, c0, c1, h, o);
+                    tmem_st32(ta, o);
+                } else if (is_sb(FMT)) {                      // the same with the high-bit plane
+                    const uint4 hd = *reinterpret_cast<const uint4*>(cs + cph);
+                    const uint4 c0 = *reinterpret_cast<const uint4*>(cs + cp0);
+                    const uint4 c1 = *reinterpret_cast<const uint4*>(cs + cp1);
+                    uint32_t pl[4];
+                    if (FMT == kFmtW6SB32) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(cs + cpp);
+                        pl[0] = v.x; pl[1] = v.y; pl[2] = v.z; pl[3] = v.w;
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2*>(cs + cpp);
+                        pl[0] = v.x; pl[1] = v.y; pl[2] = 0u; pl[3] = 0u;
+                    }
+                    uint32_t o[32];
+                    dq_sbw<FMT == kFmtW6SB32 ? 6 : 5>(hd, c0, c1, pl, h, o);
                     tmem_st32(ta, o);
                 } else if (FMT == kFmtW4G64 && KS == 256) {   // 64 weights: chunks 2h, 2h+1, one group
                     const uint4 c0 = *reinterpret_cast<const uint4*>(cs + cp0);
@@ -789,7 +872,7 @@ bool encode(EncodeTiled enc, CUtensorMap* m, CUtensorMapDataType dt, int rank, c
 
 template <int FMT, int KS, int MAXI>
 cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
-    constexpr uint32_t RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : 144;
+    constexpr uint32_t RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : sb_record(FMT);
     const EncodeTiled enc = encoder();
     if (!enc) return cudaErrorNotSupported;
     TcArgs<MAXI> p = {};
@@ -897,15 +980,18 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
 // K allows; int8 rows are 128 bytes at 128-K stages already.
 template <int FMT>
 cudaError_t launch_chunk(const WgemmArgs* a, int count, cudaStream_t st) {
-    if (FMT == kFmtW4SB32)                                  // K % 256 == 0: one record per row and stage
+    if constexpr (is_sb(FMT)) {                             // K % 256 == 0: one record per row and stage
         return count == 1 ? launch_fmt_tc<FMT, 256, 1>(a, 1, st) : launch_fmt_tc<FMT, 256, kTcMaxItems>(a, count, st);
-    if (FMT == kFmtW4G64) {
-        bool wide = a[0].M <= 64;
-        for (int i = 0; i < count; ++i) wide = wide && (a[i].K % 256 == 0);
-        if (wide)
-            return count == 1 ? launch_fmt_tc<FMT, 256, 1>(a, 1, st) : launch_fmt_tc<FMT, 256, kTcMaxItems>(a, count, st);
+    } else {
+        if (FMT == kFmtW4G64) {
+            bool wide = a[0].M <= 64;
+            for (int i = 0; i < count; ++i) wide = wide && (a[i].K % 256 == 0);
+            if (wide)
+                return count == 1 ? launch_fmt_tc<FMT, 256, 1>(a, 1, st)
+                                  : launch_fmt_tc<FMT, 256, kTcMaxItems>(a, count, st);
+        }
+        return count == 1 ? launch_fmt_tc<FMT, 128, 1>(a, 1, st) : launch_fmt_tc<FMT, 128, kTcMaxItems>(a, count, st);
     }
-    return count == 1 ? launch_fmt_tc<FMT, 128, 1>(a, 1, st) : launch_fmt_tc<FMT, 128, kTcMaxItems>(a, count, st);
 }
 
 template <int FMT>
@@ -920,14 +1006,19 @@ cudaError_t launch_chunks(const WgemmArgs* a, int count, cudaStream_t st) {
 
 }  // namespace
 
+// The 5- and 6-bit superblock formats have no register-path kernel: their
+// products run here at every M (x rows past M are zero-filled by the copy).
 bool tc_supported(int fmt, int M) {
+    if (fmt == kFmtW5SB32 || fmt == kFmtW6SB32) return M >= 1;
     return M >= kTcMinM && (fmt == kFmtW4G64 || fmt == kFmtW8G16 || fmt == kFmtW4SB32);
 }
 
 cudaError_t launch_tc(const WgemmArgs* a, int count, cudaStream_t st) {
     if (a[0].fmt == kFmtW4G64) return launch_chunks<kFmtW4G64>(a, count, st);
     if (a[0].fmt == kFmtW8G16) return launch_chunks<kFmtW8G16>(a, count, st);
-    return launch_chunks<kFmtW4SB32>(a, count, st);
+    if (a[0].fmt == kFmtW4SB32) return launch_chunks<kFmtW4SB32>(a, count, st);
+    if (a[0].fmt == kFmtW5SB32) return launch_chunks<kFmtW5SB32>(a, count, st);
+    return launch_chunks<kFmtW6SB32>(a, count, st);
 }
 
 cudaError_t status_tc(cudaStream_t st, unsigned* word) {

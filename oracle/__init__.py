@@ -9,8 +9,9 @@ CPU-baseline leg of ``bench.py`` may import this package. The product library
 The arithmetic lives in ``rq_oracle.c`` (plain C loops, IEEE fp32/fp64, no
 contraction, no fast-math); this module only compiles it and marshals numpy
 arrays. Formats are named by strings here: ``"w4g64"`` (symmetric int4, group
-64), ``"w8g16"`` (symmetric int8, group 16), ``"w4sb32"`` / ``"w5sb32"`` /
-``"w6sb32"`` (asymmetric 4-, 5-, 6-bit superblocks of 8 groups of 32).
+64), ``"w8g16"`` / ``"w8g64"`` (symmetric int8, group 16 / 64), ``"w6g16"``
+(symmetric 6-bit, group 16), ``"w4sb32"`` / ``"w5sb32"`` / ``"w6sb32"``
+(asymmetric 4-, 5-, 6-bit superblocks of 8 groups of 32).
 """
 from __future__ import annotations
 
@@ -25,11 +26,11 @@ _SRC = os.path.join(_HERE, "rq_oracle.c")
 _OUT_DIR = os.path.join(_HERE, "_build")
 _SO = os.path.join(_OUT_DIR, "librq_oracle.so")
 
-FORMATS = {"w4g64": 1, "w8g16": 2, "w4sb32": 3, "w5sb32": 4, "w6sb32": 5}
-GROUP = {"w4g64": 64, "w8g16": 16, "w4sb32": 32, "w5sb32": 32, "w6sb32": 32}
+FORMATS = {"w4g64": 1, "w8g16": 2, "w4sb32": 3, "w5sb32": 4, "w6sb32": 5, "w8g64": 6, "w6g16": 7}
+GROUP = {"w4g64": 64, "w8g16": 16, "w4sb32": 32, "w5sb32": 32, "w6sb32": 32, "w8g64": 64, "w6g16": 16}
 SB_BITS = {"w4sb32": 4, "w5sb32": 5, "w6sb32": 6}
 SB_BYTES = {"w4sb32": 144, "w5sb32": 176, "w6sb32": 208}
-QMAX = {"w4g64": 7, "w8g16": 127}
+QMAX = {"w4g64": 7, "w8g16": 127, "w8g64": 127, "w6g16": 31}
 
 _P = ctypes.c_void_p
 _i = ctypes.c_int
@@ -208,6 +209,10 @@ def packed_shapes(fmt: str, K: int, N: int):
         return (N, K // 2), np.uint8, (N, K // 64)
     if fmt == "w8g16":
         return (N, K), np.uint8, (N, K // 16)
+    if fmt == "w8g64":
+        return (N, K), np.uint8, (N, K // 64)
+    if fmt == "w6g16":
+        return (N, K // 64 * 48), np.uint8, (N, K // 16)
     if fmt in SB_BYTES:
         return (N, (K // 256) * SB_BYTES[fmt]), np.uint8, None
     raise ValueError(fmt)

@@ -50,6 +50,12 @@
 #define ORC_W4SB32 3
 #define ORC_W5SB32 4
 #define ORC_W6SB32 5
+#define ORC_W8G64 6
+#define ORC_W6G16 7
+
+/* Bits per code and group size of the symmetric formats. */
+static int sym_bits(int fmt) { return fmt == ORC_W4G64 ? 4 : (fmt == ORC_W6G16 ? 6 : 8); }
+static int sym_gsize(int fmt) { return (fmt == ORC_W4G64 || fmt == ORC_W8G64) ? 64 : 16; }
 
 /* Bits per code and record bytes of the superblock formats (4, 5, 6 bits:
  * 144, 176, 208 bytes per 256 weights). */
@@ -214,12 +220,23 @@ int orc_sym_group(const float *w, const float *a, int G, int qmax,
  *                  scales [N][K/64] fp16.                         ([CARD])
  *   int8 group 16: codes [N][K] bytes, byte = q + 128; scales [N][K/16] fp16.
  *                                                                   ([ART])
+ *   int8 group 64: the int8 codes with scales [N][K/64] fp16 (the int8 tier
+ *                  of the model card's format list).
+ *   6-bit group 16 (REDUCTION preset's channel-mix, [ART]): qmax = 31,
+ *                  u = q + 32 in [1, 63]; codes [N][K/64 * 48] bytes, one
+ *                  48-byte chunk per 64 weights j = 0..63 of a row:
+ *                    bytes [0:32]  low 4 bits of u_j: byte j/2, low nibble for
+ *                                  even j, high nibble for odd j
+ *                    bytes [32:48] bits 4..5 of u_j in bits 2 (j % 4) .. +1
+ *                                  of byte 32 + j/4
+ *                  scales [N][K/16] fp16. 7 bits per weight. The layout is
+ *                  this project's own (the pages give only the bit width).
  * a == NULL means every a_k = 1 (plain MSE search). */
 void orc_pack_sym(const float *W, int K, int N, const float *a, int fmt,
                   int n_cand, float t_lo, float t_hi, uint8_t *codes, uint16_t *scales)
 {
-    int bits = (fmt == ORC_W4G64) ? 4 : 8;
-    int G = (fmt == ORC_W4G64) ? 64 : 16;
+    int bits = sym_bits(fmt);
+    int G = sym_gsize(fmt);
     int qmax = (1 << (bits - 1)) - 1;
     int ng = K / G;
     float *t = (float *)malloc(sizeof(float) * (size_t)n_cand);
@@ -237,6 +254,14 @@ void orc_pack_sym(const float *W, int K, int N, const float *a, int fmt,
                 size_t kk = (size_t)g * G + k;
                 if (bits == 8) {
                     codes[(size_t)n * K + kk] = (uint8_t)(q[k] + 128);
+                } else if (bits == 6) {
+                    int u = q[k] + 32;
+                    uint8_t *chunk = codes + (size_t)n * (K / 64 * 48) + (kk / 64) * 48;
+                    size_t j = kk % 64;
+                    if ((j & 1) == 0) chunk[j / 2] = (uint8_t)(u & 15);
+                    else chunk[j / 2] = (uint8_t)(chunk[j / 2] | ((u & 15) << 4));
+                    if (j % 4 == 0) chunk[32 + j / 4] = 0;
+                    chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (2 * (j % 4)));
                 } else {
                     uint8_t u = (uint8_t)(q[k] + 8);
                     uint8_t *byte = codes + (size_t)n * (K / 2) + kk / 2;
@@ -442,12 +467,21 @@ static void deq_row(int fmt, int K, const uint8_t *codes, const uint16_t *scales
         }
         return;
     }
-    int G = (fmt == ORC_W4G64) ? 64 : 16;
+    int G = sym_gsize(fmt);
     int ng = K / G;
     for (int k = 0; k < K; k++) {
         int q;
-        if (fmt == ORC_W4G64) q = ((codes[(size_t)n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xf) - 8;
-        else q = (int)codes[(size_t)n * K + k] - 128;
+        if (fmt == ORC_W4G64) {
+            q = ((codes[(size_t)n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xf) - 8;
+        } else if (fmt == ORC_W6G16) {
+            const uint8_t *chunk = codes + (size_t)n * (K / 64 * 48) + (k / 64) * 48;
+            int j = k % 64;
+            int u = (chunk[j / 2] >> (4 * (j & 1))) & 0xf;
+            u |= ((chunk[32 + j / 4] >> (2 * (j % 4))) & 3) << 4;
+            q = u - 32;
+        } else {
+            q = (int)codes[(size_t)n * K + k] - 128;
+        }
         float s = orc_f16_to_f32(scales[(size_t)n * ng + k / G]);
         out[k] = (float)q * s;
     }

@@ -37,6 +37,13 @@ MUTANTS = [
      "float s = orc_f16_to_f32(scales[(size_t)n * ng]);", None),
     ("sb dequant adds the min", "float p = (float)q * S;\n    return p - M;", "float p = (float)q * S;\n    return p + M;", None),
     ("absmax from the last element", "if (v > absmax) absmax = v;", "absmax = v;", None),
+    ("6-bit symmetric plane bit order", "chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (2 * (j % 4)));",
+     "chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (6 - 2 * (j % 4)));", None),
+    ("6-bit symmetric code offset 31", "int u = q[k] + 32;", "int u = q[k] + 31;", None),
+    ("6-bit symmetric low nibbles swapped", "if ((j & 1) == 0) chunk[j / 2] = (uint8_t)(u & 15);",
+     "if ((j & 1) == 1) chunk[j / 2] = (uint8_t)(u & 15);", None),
+    ("int8 g64 search on the first 16 weights", "orc_sym_group(row + (size_t)g * G, a ? a + (size_t)g * G : NULL, G, qmax,",
+     "orc_sym_group(row + (size_t)g * G, a ? a + (size_t)g * G : NULL, G == 64 && bits == 8 ? 16 : G, qmax,", None),
     ("E[x^2] sums |x| instead of x^2", "part = part + v * v;", "part = part + fabs(v);", None),
     ("E[x^2] skips the last chunk", "for (int c = 0; c < 64; c++) {\n            int r0", "for (int c = 0; c < 63; c++) {\n            int r0", None),
     ("E[x^2] divides by rows - 1", "act_sq[k] = (float)(sum_sq[k] / (double)rows);", "act_sq[k] = (float)(sum_sq[k] / (double)(rows - 1));", None),

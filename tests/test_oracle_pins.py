@@ -174,7 +174,7 @@ def test_sym_ties_pick_lowest_index(orc):
 
 
 # ---------------------------------------------------- RTN closed form ------
-@pytest.mark.parametrize("fmt", ["w4g64", "w8g16"])
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w8g64", "w6g16"])
 def test_rtn_error_at_most_half_scale(orc, fmt):
     """RTN (one candidate, t = 1): no code clamps, every element is within
     s/2 of its dequantized value, and each group's absmax maps to +-qmax."""
@@ -196,7 +196,7 @@ def test_rtn_error_at_most_half_scale(orc, fmt):
 
 
 # ----------------------------------------------------------- invariants ----
-@pytest.mark.parametrize("fmt", ["w4g64", "w8g16"])
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w8g64", "w6g16"])
 def test_sym_invariants(orc, fmt):
     G = orc.GROUP[fmt]
     rng = np.random.default_rng(9)
@@ -211,7 +211,7 @@ def test_sym_invariants(orc, fmt):
     assert np.array_equal(orc.dequant(fmt, 256, 4, c1, s1), -q0)
     # W -> 2^e W: same codes, scales x 2^e, while every scale stays an fp16
     # normal (below 2^-14 the fp16 grid is coarser and the invariant is void)
-    for e in ((-3, 2) if fmt == "w4g64" else (1, 3)):
+    for e in {"w4g64": (-3, 2), "w6g16": (-2, 2)}.get(fmt, (1, 3)):
         sc = np.ldexp(orc.f16_bits_to_f32(s0), e)
         assert np.all(sc >= 2.0 ** -14) and np.all(sc <= 60000.0)
         c2, s2 = orc.pack(fmt, np.ldexp(W, e).astype(np.float32), a)
@@ -255,7 +255,8 @@ def designed_sym(rng, N, K, G, qmax, unit):
     return q, (q * unit).astype(np.float32)
 
 
-@pytest.mark.parametrize("fmt,unit", [("w4g64", 2.0 ** -6), ("w8g16", 2.0 ** -10)])
+@pytest.mark.parametrize("fmt,unit", [("w4g64", 2.0 ** -6), ("w8g16", 2.0 ** -10), ("w8g64", 2.0 ** -10),
+                                      ("w6g16", 2.0 ** -8)])
 @pytest.mark.parametrize("n_cand", [1, 64])
 def test_exact_products_sym(orc, fmt, unit, n_cand):
     """w = q * 2^-e with each group's absmax at qmax * 2^-e: the scale is 2^-e
@@ -274,6 +275,36 @@ def test_exact_products_sym(orc, fmt, unit, n_cand):
     xb = (xi.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
     y = orc.wgemm(fmt, xb, K, N, codes, scales)
     assert np.array_equal(y, (xi @ q.T).astype(np.float64) * unit)
+
+
+def test_w6g16_bytes_follow_the_layout(orc):
+    """The 6-bit symmetric codes, read back from the bytes by the layout's
+    definition (per 64 weights: 32 bytes of low nibbles, even j in the low
+    half of byte j/2; then bits 4..5 of u_j at bits 2 (j % 4) of byte
+    32 + j/4), are u = q + 32 for weights built as q * 2^-8 with every
+    group's absmax at 31 * 2^-8."""
+    rng = np.random.default_rng(37)
+    N, K = 6, 320
+    q, W = designed_sym(rng, N, K, 16, 31, 2.0 ** -8)
+    codes, scales = orc.pack("w6g16", W, None, n_cand=1)
+    assert codes.shape == (N, K // 64 * 48)
+    assert np.all(orc.f16_bits_to_f32(scales) == np.float32(2.0 ** -8))
+    u = np.zeros((N, K), dtype=np.int64)
+    for n in range(N):
+        for k in range(K):
+            ch = codes[n, (k // 64) * 48:(k // 64) * 48 + 48].astype(np.int64)
+            j = k % 64
+            lo = (ch[j // 2] >> (4 * (j % 2))) & 15
+            hi = (ch[32 + j // 4] >> (2 * (j % 4))) & 3
+            u[n, k] = lo + 16 * hi
+    assert np.array_equal(u, q + 32)
+
+
+def test_sym_bits_per_weight(orc):
+    """Stored bits per weight: codes plus one fp16 scale per group."""
+    K = N = 4096
+    for fmt, bpw in [("w4g64", 4.25), ("w8g16", 9.0), ("w8g64", 8.25), ("w6g16", 7.0)]:
+        assert packed_bytes(orc, fmt, K, N) * 8 / (K * N) == bpw
 
 
 def test_exact_products_sb32(orc):
@@ -450,7 +481,7 @@ def test_asym_t1_covers_the_group_range(orc, bits):
 
 
 # ------------------------------------------------ reduction to a library ----
-@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w4sb32"])
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w4sb32", "w8g64", "w6g16", "w5sb32"])
 def test_product_matches_numpy_matmul(orc, fmt):
     rng = np.random.default_rng(71)
     N, K, M = 40, 768, 5

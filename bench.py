@@ -257,7 +257,7 @@ class Problem:
             for i in range(0, len(cs), rq.MAX_BATCH):
                 ch = cs[i:i + rq.MAX_BATCH]
                 self.batches.append(rq.WgemmBatch([c[0] for c in ch], [c[1] for c in ch], [c[2] for c in ch]))
-                tc = M >= rq.TC_MIN_M and fmt in ("w4g64", "w8g16")
+                tc = rq.tc_path(fmt, M)
                 self.kernel_launches += -(-len(ch) // rq.TC_MAX_ITEMS) if tc else 1
         torch.cuda.synchronize()
 
@@ -399,33 +399,42 @@ def run_ours(args, w, M):
     # workload at its other M, and the other four configurations), one
     # batched step per (configuration, M)
     from weight_only_quantized_rq_b200 import workloads as wl
-    configs = {}
+    def measure(w2, mats2, Ms):
+        entry = {"workload": w2.name, "packed_bytes_per_step": sum(p.nbytes for _, _, p in mats2)}
+        for m2 in Ms:
+            pr = Problem(w2, mats2, m2, dev)
+            f = capture(lambda pr=pr: pr.step(stream))
+            ms2 = timed(f, min(args.steps, 10))
+            t_roof = pr.roofline_s(hbm, tc_peak)
+            entry[str(m2)] = {
+                "ms_per_step": round(ms2, 5),
+                "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
+                "pct_hbm_measured": round(100 * pr.packed_bytes / (ms2 * 1e-3) / 1e9 / hbm, 2),
+                "TFLOP_s": round(ws * pr.flops / (ms2 * 1e-3) / 1e12, 2),
+                "pct_bf16_peak_measured": round(100 * pr.flops / (ms2 * 1e-3) / 1e12 / tc_peak, 2),
+                "roofline_frac": round(t_roof / (ms2 * 1e-3), 4),
+                "launches_per_step": pr.kernel_launches,
+                "kernel": "tc_kernel" if all(rq.tc_path(c[3].fmt, m2) for c in pr.calls) else "gemv_kernel"}
+            del pr
+        return entry
+
+    configs, variants = {}, {}
     if not args.quick:
         for wi, w2 in enumerate(wl.WORKLOADS):
             Ms = [m for m in w2.Ms if not (w2 is w and m == M)]
             if not Ms:
                 continue
             mats2 = mats if w2 is w else pack_workload(w2, dev)
-            entry = {"workload": w2.name, "packed_bytes_per_step": sum(p.nbytes for _, _, p in mats2)}
-            for m2 in Ms:
-                pr = Problem(w2, mats2, m2, dev)
-                f = capture(lambda pr=pr: pr.step(stream))
-                ms2 = timed(f, min(args.steps, 10))
-                t_roof = pr.roofline_s(hbm, tc_peak)
-                entry[str(m2)] = {
-                    "ms_per_step": round(ms2, 5),
-                    "GB_s": round(ws * pr.packed_bytes / (ms2 * 1e-3) / 1e9, 2),
-                    "pct_hbm_measured": round(100 * pr.packed_bytes / (ms2 * 1e-3) / 1e9 / hbm, 2),
-                    "TFLOP_s": round(ws * pr.flops / (ms2 * 1e-3) / 1e12, 2),
-                    "pct_bf16_peak_measured": round(100 * pr.flops / (ms2 * 1e-3) / 1e12 / tc_peak, 2),
-                    "roofline_frac": round(t_roof / (ms2 * 1e-3), 4),
-                    "launches_per_step": pr.kernel_launches,
-                    "kernel": "gemv_kernel" if m2 < rq.TC_MIN_M else "tc_kernel"}
-                del pr
-            configs[f"config{wi + 1}"] = entry
+            configs[f"config{wi + 1}"] = measure(w2, mats2, Ms)
             if w2 is not w:
                 del mats2
                 torch.cuda.empty_cache()
+        # the preset's wider-code matrices (5- and 6-bit superblocks)
+        for w2 in wl.VARIANTS:
+            mats2 = pack_workload(w2, dev)
+            variants[w2.name.split(" ")[0] + "/" + w2.per_layer[0].name] = measure(w2, mats2, list(w2.Ms))
+            del mats2
+            torch.cuda.empty_cache()
     # the E[x^2] statistic of the scale search over a calibration batch of
     # 7.2B width (32768 rows x 4096 channels of bf16, 256 MB > L2)
     act_stats = None
@@ -466,6 +475,7 @@ def run_ours(args, w, M):
         "configs_note": "per (configuration, M): one graph-captured step of batched launches over the "
                         "configuration's products; roofline_frac = sum over products of max(bytes / HBM peak, "
                         "flops / bf16 peak) divided by the step time",
+        "preset_variants": variants,
         "act_stats": act_stats,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": prob.h2d,

@@ -67,6 +67,17 @@ typedef enum rq_status {
  *   codes  [N][K] bytes, byte = q + 128, q in [-127, 127].
  *   scales [N][K/16] fp16.   w_hat = q * scale. 9 bits per weight.
  *
+ * RQ_W8_SYM_G64 ([CARD] "Accuracy warning": the int8 w8g64 tier it recommends
+ *   for reasoning-heavy use): RQ_W8_SYM_G16 with groups of 64: scales
+ *   [N][K/64] fp16. 8.25 bits per weight.
+ *
+ * RQ_W6_SYM_G16 ([ART], the REDUCTION preset's channel-mix in 6 bits):
+ *   symmetric, group 16, q in [-31, 31], u = q + 32 in [1, 63].
+ *   codes  [N][K/64 * 48] bytes, one 48-byte chunk per 64 weights j = 0..63:
+ *          [0:32]  low 4 bits of u_j: byte j/2, low nibble for even j
+ *          [32:48] bits 4..5 of u_j in bits 2 (j % 4) .. +1 of byte 32 + j/4
+ *   scales [N][K/16] fp16.   w_hat = q * scale. 7 bits per weight.
+ *
  * RQ_W4_ASYM_SB32 ([ART], COMPRESSION projections): asymmetric int4 in
  *   superblocks of 256 weights = 8 groups of 32 along K; one 144-byte record
  *   per superblock, records [N][K/256]:
@@ -94,7 +105,9 @@ typedef enum rq_format {
     RQ_W8_SYM_G16 = 2,
     RQ_W4_ASYM_SB32 = 3,
     RQ_W5_ASYM_SB32 = 4,
-    RQ_W6_ASYM_SB32 = 5
+    RQ_W6_ASYM_SB32 = 5,
+    RQ_W8_SYM_G64 = 6,
+    RQ_W6_SYM_G16 = 7
 } rq_format;
 
 /* Candidate grid of the E[x^2]-weighted search ([ART]): n_cand points
@@ -137,7 +150,7 @@ size_t rq_packed_size(int fmt, int K, int N, size_t *codes_bytes, size_t *scales
  *   out    descriptor whose fmt/K/N must equal the call's and whose planes
  *          receive the codes and scales.
  * For each symmetric group: absmax = max|w|, base = absmax / qmax (fp32,
- * qmax = 7 or 127); candidate i has scale s_i = fp16(t_i * base); its loss is
+ * qmax = 7, 31 or 127); candidate i has scale s_i = fp16(t_i * base); its loss is
  * sum_k a_k (w_k - q_k s_i)^2 with q_k = clamp(rint(w_k / s_i), -qmax, qmax),
  * evaluated in fp64 in ascending k; the lowest index attaining the minimum
  * wins. For each asymmetric group of 32: lo = min(0, min w),
@@ -161,8 +174,9 @@ int rq_quantize_pack(const float *W, int K, int N, const float *act_sq,
  *   w   packed matrix
  *   y   device fp32 [M][N], overwritten (not accumulated into)
  * w_hat is formed in registers (M <= 2: CUDA-core GEMV, exact fp32 w_hat) or
- * in tensor memory (M >= 3, and every M for the 5- and 6-bit formats:
- * tensor-core kernel, w_hat rounded once to bf16)
+ * in tensor memory (M >= 3, and every M for the 5- and 6-bit formats
+ * RQ_W5/W6_ASYM_SB32 and RQ_W6_SYM_G16: tensor-core kernel, w_hat rounded
+ * once to bf16)
  * and never written out; the products accumulate in fp32. Kernels are launched with programmatic
  * dependent launch allowed: they read the packed weights while the kernel
  * launched just before them on the stream may still be running, and read x

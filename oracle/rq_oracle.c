@@ -220,8 +220,8 @@ int orc_sym_group(const float *w, const float *a, int G, int qmax,
  *                  scales [N][K/64] fp16.                         ([CARD])
  *   int8 group 16: codes [N][K] bytes, byte = q + 128; scales [N][K/16] fp16.
  *                                                                   ([ART])
- *   int8 group 64: the int8 codes with scales [N][K/64] fp16 (the int8 tier
- *                  of the model card's format list).
+ *   int8 group 64: the int8 codes with scales [N][K/64] fp16 (the int8 w8g64
+ *                  tier that [CARD] "Accuracy warning" recommends).
  *   6-bit group 16 (REDUCTION preset's channel-mix, [ART]): qmax = 31,
  *                  u = q + 32 in [1, 63]; codes [N][K/64 * 48] bytes, one
  *                  48-byte chunk per 64 weights j = 0..63 of a row:

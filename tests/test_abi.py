@@ -47,26 +47,31 @@ def test_version_and_status_strings(L):
     ("w4sb32", 2560, 2560, 2560 * 10 * 144, 0),
     ("w5sb32", 2560, 2560, 2560 * 10 * 176, 0),
     ("w6sb32", 256, 3, 3 * 208, 0),
+    ("w8g64", 2048, 5, 5 * 2048, 5 * 32 * 2),
+    ("w6g16", 320, 3, 3 * 5 * 48, 128),     # 3 rows x 20 scales x 2 B = 120, padded to 128
     ("w4g64", 768, 3, 3 * 384, 80),        # 3 rows x 12 scales x 2 B = 72, padded to 80
 ])
 def test_packed_size(L, fmt, K, N, codes, scales):
     cb, sb = rq.rq_packed_size(fmt, K, N)
     assert cb == codes
-    raw = N * (K // 64) * 2 if fmt == "w4g64" else (N * (K // 16) * 2 if fmt == "w8g16" else 0)
+    G = {"w4g64": 64, "w8g64": 64, "w8g16": 16, "w6g16": 16}.get(fmt)
+    raw = N * (K // G) * 2 if G else 0
     assert sb == (raw + 15) // 16 * 16
     assert sb == scales
 
 
 def test_bits_per_weight(L):
     K = N = 4096
-    for fmt, bpw in [("w4g64", 4.25), ("w8g16", 9.0), ("w4sb32", 4.5), ("w5sb32", 5.5), ("w6sb32", 6.5)]:
+    for fmt, bpw in [("w4g64", 4.25), ("w8g16", 9.0), ("w4sb32", 4.5), ("w5sb32", 5.5), ("w6sb32", 6.5),
+                     ("w8g64", 8.25), ("w6g16", 7.0)]:
         cb, sb = rq.rq_packed_size(fmt, K, N)
         assert (cb + sb) * 8 / (K * N) == bpw
 
 
 @pytest.mark.parametrize("fmt,K,N", [("w4g64", 96, 4), ("w4sb32", 320, 4), ("w8g16", 65536, 4),
                                      ("w5sb32", 320, 4), ("w6sb32", 64, 4), ("w4g64", 2048, 0),
-                                     ("w4g64", 32, 1), (7, 2048, 2), (6, 2048, 2), (0, 2048, 2)])
+                                     ("w8g64", 96, 4), ("w6g16", 32, 4),
+                                     ("w4g64", 32, 1), (8, 2048, 2), (0, 2048, 2)])
 def test_packed_size_rejects(L, fmt, K, N):
     f = rq.fmt_id(fmt)
     assert L.rq_packed_size(f, K, N, None, None) == 0

@@ -73,7 +73,7 @@ def test_guard_band_and_padding():
     assert bool((big[:32] == 7.0).all()) and bool((big[32 + K:] == 7.0).all())
 
 
-@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w4sb32", "w5sb32", "w6sb32"])
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w4sb32", "w5sb32", "w6sb32", "w8g64", "w6g16"])
 def test_calibrate_then_pack_matches_oracle_chain(fmt):
     """Device statistic -> device pack gives the codes of oracle statistic ->
     oracle pack: the whole calibration path stays on the GPU."""

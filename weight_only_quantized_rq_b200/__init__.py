@@ -7,10 +7,11 @@ streams; every step of the computation runs in librq's CUDA kernels. There is
 no fallback: if librq.so is missing, every call raises.
 
 Formats (see include/rq.h): ``RQ_W4_SYM_G64`` (symmetric int4, group 64),
-``RQ_W8_SYM_G16`` (symmetric int8, group 16), ``RQ_W4_ASYM_SB32``,
+``RQ_W8_SYM_G16`` / ``RQ_W8_SYM_G64`` (symmetric int8, group 16 / 64),
+``RQ_W6_SYM_G16`` (symmetric 6-bit, group 16), ``RQ_W4_ASYM_SB32``,
 ``RQ_W5_ASYM_SB32``, ``RQ_W6_ASYM_SB32`` (asymmetric 4-, 5-, 6-bit superblocks
-of 8 groups of 32). The strings "w4g64", "w8g16", "w4sb32", "w5sb32",
-"w6sb32" are accepted wherever a format is expected.
+of 8 groups of 32). The strings "w4g64", "w8g16", "w8g64", "w6g16", "w4sb32",
+"w5sb32", "w6sb32" are accepted wherever a format is expected.
 """
 from __future__ import annotations
 
@@ -36,16 +37,28 @@ RQ_W8_SYM_G16 = 2
 RQ_W4_ASYM_SB32 = 3
 RQ_W5_ASYM_SB32 = 4
 RQ_W6_ASYM_SB32 = 5
+RQ_W8_SYM_G64 = 6
+RQ_W6_SYM_G16 = 7
 FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_ASYM_SB32,
-              "w5sb32": RQ_W5_ASYM_SB32, "w6sb32": RQ_W6_ASYM_SB32}
+              "w5sb32": RQ_W5_ASYM_SB32, "w6sb32": RQ_W6_ASYM_SB32, "w8g64": RQ_W8_SYM_G64,
+              "w6g16": RQ_W6_SYM_G16}
 SB_FORMATS = (RQ_W4_ASYM_SB32, RQ_W5_ASYM_SB32, RQ_W6_ASYM_SB32)
 EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_dequant",
            "rq_act_sumsq", "rq_act_finalize",
            "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
 MAX_BATCH = 160
 TC_MIN_M = 3         # activation rows from which int4/int8/4-bit superblock products run on the tensor cores
-                     # (5- and 6-bit superblock products run there at every M)
+                     # (5- and 6-bit products run there at every M)
 TC_MAX_ITEMS = 96    # products per tensor-core launch (larger batches take several)
+
+
+def tc_path(fmt, M: int) -> bool:
+    """Whether products of this format at M activation rows run on the
+    tensor-core kernel (else on the register-path GEMV)."""
+    f = fmt_id(fmt)
+    if f in (RQ_W5_ASYM_SB32, RQ_W6_ASYM_SB32, RQ_W6_SYM_G16):
+        return True
+    return M >= TC_MIN_M
 
 
 class RqSearch(ctypes.Structure):

@@ -13,7 +13,9 @@ namespace {
 
 thread_local int t_last_cuda = 0;
 
-bool fmt_ok(int fmt) { return fmt == rq::kFmtW4G64 || fmt == rq::kFmtW8G16 || rq::is_sb(fmt); }
+bool fmt_ok(int fmt) {
+    return fmt == rq::kFmtW4G64 || rq::is_w8(fmt) || fmt == rq::kFmtW6G16 || rq::is_sb(fmt);
+}
 
 // RQ_OK, or the status for an unsupported (fmt, K, N).
 int shape_status(int fmt, int K, int N) {

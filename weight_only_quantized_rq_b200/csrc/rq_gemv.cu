@@ -106,7 +106,7 @@ __device__ __forceinline__ void item_units(const Item& it, long long lo, long lo
 // (fp16 for the int4 formats, fp32 for int8), then for the int4 formats a
 // metadata record per row m and half-chunk h (g64: float2, sb32: float4).
 __host__ __device__ constexpr size_t xvals_bytes(int fmt, int K, int MT) {
-    return (size_t)MT * K * (fmt != kFmtW8G16 ? 2 : 4);
+    return (size_t)MT * K * (!is_w8(fmt) ? 2 : 4);
 }
 __host__ __device__ constexpr size_t xbuf_bytes(int fmt, int K, int MT) {
     return xvals_bytes(fmt, K, MT) + (size_t)MT * (fmt == kFmtW4G64 ? (K / 64) * 8 : fmt == kFmtW4SB32 ? (K / 32) * 16 : 0);
@@ -155,7 +155,7 @@ constexpr int kCoopBarrier = 15;
 
 template <int FMT, int MT>
 __device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xb, int first, int stride) {
-    constexpr bool kW4 = FMT != kFmtW8G16;
+    constexpr bool kW4 = !is_w8(FMT);
     const int hcpr = it.K >> 5, n = MT * hcpr;
     uint8_t* meta = xb + xvals_bytes(FMT, it.K, MT);
     if constexpr (FMT == kFmtW4G64) {
@@ -258,7 +258,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& c, int i) {
 template <int FMT, int MT, int RW, int TT>
 __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s, int m0, int mrows, int lane, int rbase, int slice,
                                            float* red) {
-    constexpr bool kW4 = FMT != kFmtW8G16;
+    constexpr bool kW4 = !is_w8(FMT);
     constexpr int U = RW == 1 ? 2 : 1;                   // half-chunks per iteration
     const int hcpr = it.K >> 5, T = TT ? TT : it.T, HJ = it.HJ;   // TT: team lanes fixed at compile time
     const int li = lane & (T - 1);
@@ -390,13 +390,14 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             }
         }
     } else {
-        // int8 group 16: 32 code bytes per row and half-chunk = groups 2h, 2h+1;
-        // x as fp32 quads, 8 per half-chunk
+        // int8: 32 code bytes per row and half-chunk h = groups 2h, 2h+1 of
+        // 16 (two scales) or half of group h/2 of 64 (one scale); x as fp32
+        // quads, 8 per half-chunk
         uint32_t ca[RW], sa[RW];
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
             ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)li * 32u;
-            sa[r] = ssc_s + (uint32_t)(rbase + r) * srb + (uint32_t)li * 4u;
+            sa[r] = ssc_s + (uint32_t)(rbase + r) * srb;
         }
         for (int hj = 0; hj < HJ; hj += U) {
 #pragma unroll
@@ -407,7 +408,9 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
                 for (int r = 0; r < RW; ++r) {
                     const uint4 c0 = lds128_a(ca[r] + dh * 32u);
                     const uint4 c1 = lds128_a(ca[r] + dh * 32u + 16u);
-                    const uint32_t sp = lds32_a(sa[r] + dh * 4u);
+                    const uint32_t hc = dh + (uint32_t)li;   // this lane's half-chunk of the row
+                    const uint32_t sp = FMT == kFmtW8G64 ? lds16_a(sa[r] + ((hc >> 1) << 1)) * 0x10001u
+                                                         : lds32_a(sa[r] + hc * 4u);
                     const float s0 = __half2float(__ushort_as_half((unsigned short)(sp & 0xffffu)));
                     const float s1 = __half2float(__ushort_as_half((unsigned short)(sp >> 16)));
 #pragma unroll
@@ -898,8 +901,9 @@ cudaError_t launch_gemv(const WgemmArgs* a, int count, cudaStream_t st) {
     switch (a[0].fmt) {
         case kFmtW4G64: return launch_fmt<kFmtW4G64>(a, count, st);
         case kFmtW8G16: return launch_fmt<kFmtW8G16>(a, count, st);
+        case kFmtW8G64: return launch_fmt<kFmtW8G64>(a, count, st);
         case kFmtW4SB32: return launch_fmt<kFmtW4SB32>(a, count, st);
-        default: return cudaErrorNotSupported;            // 5- and 6-bit records run on the tensor-core kernel
+        default: return cudaErrorNotSupported;            // 5- and 6-bit codes run on the tensor-core kernel
     }
 }
 

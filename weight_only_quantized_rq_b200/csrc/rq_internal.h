@@ -13,6 +13,13 @@ constexpr int kFmtW8G16 = 2;
 constexpr int kFmtW4SB32 = 3;
 constexpr int kFmtW5SB32 = 4;
 constexpr int kFmtW6SB32 = 5;
+constexpr int kFmtW8G64 = 6;
+constexpr int kFmtW6G16 = 7;
+
+// int8 codes (one byte per weight; group 16 or 64).
+__host__ __device__ constexpr bool is_w8(int fmt) { return fmt == kFmtW8G16 || fmt == kFmtW8G64; }
+// Weights per fp16 scale of the symmetric formats.
+__host__ __device__ constexpr int sym_group(int fmt) { return fmt == kFmtW4G64 || fmt == kFmtW8G64 ? 64 : 16; }
 
 // The asymmetric superblock formats: bits per code and bytes per record of
 // 256 weights (16-byte header, 128 bytes of low nibbles, high-bit plane).
@@ -22,11 +29,16 @@ __host__ __device__ constexpr int sb_record(int fmt) { return 16 + 128 + (sb_bit
 
 // Bytes per row of the codes plane (records plane for the superblock formats)
 // and of the scales plane.
+// 6-bit symmetric codes: 48 bytes per 64 weights (32 bytes of low nibbles,
+// then 16 bytes of the codes' bits 4..5).
 inline size_t code_row_bytes(int fmt, int K) {
-    return fmt == kFmtW4G64 ? (size_t)K / 2 : fmt == kFmtW8G16 ? (size_t)K : (size_t)K / 256 * sb_record(fmt);
+    return fmt == kFmtW4G64 ? (size_t)K / 2
+         : is_w8(fmt)       ? (size_t)K
+         : fmt == kFmtW6G16 ? (size_t)K / 64 * 48
+                            : (size_t)K / 256 * sb_record(fmt);
 }
 inline size_t scale_row_bytes(int fmt, int K) {
-    return fmt == kFmtW4G64 ? (size_t)K / 32 : fmt == kFmtW8G16 ? (size_t)K / 8 : 0;
+    return is_sb(fmt) ? 0 : (size_t)K / sym_group(fmt) * 2;
 }
 __host__ __device__ inline size_t round16(size_t v) { return (v + 15) & ~(size_t)15; }
 
@@ -59,8 +71,9 @@ struct WgemmArgs {
 constexpr int kMaxBatch = 160;
 cudaError_t launch_gemv(const WgemmArgs* a, int count, cudaStream_t st);
 
-// Tensor-core path (kTcMinM <= M <= 128; int4 g64 and int8 g16): bf16 tiles
-// dequantized into tensor memory, tcgen05.mma against x in shared memory.
+// Tensor-core path (kTcMinM <= M <= 128; every M for the 5- and 6-bit
+// formats): bf16 tiles dequantized into tensor memory, tcgen05.mma against x
+// in shared memory.
 // `count` independent products of one format and one M share a launch.
 constexpr int kTcMinM = 3;
 bool tc_supported(int fmt, int M);

@@ -60,8 +60,9 @@ __device__ __forceinline__ void warp_argmin(double& L, int& idx) {
 constexpr int kPackWarps = 8;
 constexpr double kInf = __builtin_huge_val();
 
-// One warp per symmetric group of G weights (G = 64: int4, qmax 7;
-// G = 16: int8, qmax 127). Lane l evaluates candidates l, l+32, ...
+// One warp per symmetric group of G weights: int4 (G = 64, qmax 7), int8
+// (G = 16 or 64, qmax 127), 6-bit (G = 16, qmax 31). Lane l evaluates
+// candidates l, l+32, ...
 template <int G, int QMAX>
 __global__ void __launch_bounds__(kPackWarps * 32)
 qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
@@ -111,15 +112,33 @@ qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restr
         best_s = __float2half_rn(__fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), base));
     }
     const float sf = __half2float(best_s);
-    if (G == 64) {
+    if (QMAX == 7) {
         // lane l writes byte l of the group: k = 2l (low nibble), 2l+1 (high)
         const int q0 = sym_code(s_w[warp][2 * lane], sf, qmax);
         const int q1 = sym_code(s_w[warp][2 * lane + 1], sf, qmax);
         codes[(size_t)n * (K / 2) + (size_t)g * 32 + lane] = (uint8_t)((q0 + 8) | ((q1 + 8) << 4));
+    } else if (QMAX == 127) {
+        for (int k = lane; k < G; k += 32) {
+            const int q = sym_code(s_w[warp][k], sf, qmax);
+            codes[(size_t)n * K + (size_t)g * G + k] = (uint8_t)(q + 128);
+        }
     } else {
-        if (lane < G) {
-            const int q = sym_code(s_w[warp][lane], sf, qmax);
-            codes[(size_t)n * K + (size_t)g * G + lane] = (uint8_t)(q + 128);
+        // 6 bits, u = q + 32: group g is weights j0 .. j0 + 15 of the 64-weight
+        // chunk g / 4 (j0 = 16 (g % 4)); lanes 0..7 write its low-nibble bytes
+        // (weights j0 + 2l, j0 + 2l + 1), lanes 8..11 its plane bytes (bits 4..5
+        // of weights j0 + 4i .. j0 + 4i + 3)
+        uint8_t* chunk = codes + (size_t)n * (K / 64 * 48) + (size_t)(g >> 2) * 48;
+        const int j0 = 16 * (g & 3);
+        if (lane < 8) {
+            const int u0 = sym_code(s_w[warp][2 * lane], sf, qmax) + 32;
+            const int u1 = sym_code(s_w[warp][2 * lane + 1], sf, qmax) + 32;
+            chunk[j0 / 2 + lane] = (uint8_t)((u0 & 15) | ((u1 & 15) << 4));
+        } else if (lane < 12) {
+            const int i = lane - 8;
+            uint32_t v = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v |= (uint32_t)((sym_code(s_w[warp][4 * i + e], sf, qmax) + 32) >> 4) << (2 * e);
+            chunk[32 + j0 / 4 + i] = (uint8_t)v;
         }
     }
     if (lane == 0) scales[(size_t)n * ng + g] = __half_as_ushort(best_s);
@@ -283,6 +302,7 @@ __global__ void dequant_w4_kernel(const uint32_t* __restrict__ codes, const __ha
     dst[1] = make_float4(o[4], o[5], o[6], o[7]);
 }
 
+template <int G>
 __global__ void dequant_w8_kernel(const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
                                   int K, long long words, float* __restrict__ out) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -290,11 +310,36 @@ __global__ void dequant_w8_kernel(const uint32_t* __restrict__ codes, const __ha
     const long long wpr = K / 4;
     const long long n = i / wpr;
     const int k0 = (int)(i % wpr) * 4;
-    const float s = __half2float(scales[n * (K / 16) + k0 / 16]);
+    const float s = __half2float(scales[n * (K / G) + k0 / G]);
     float f[4];
     unpack_w8(codes[i], f);
     *reinterpret_cast<float4*>(out + n * K + k0) =
         make_float4(__fmul_rn(f[0], s), __fmul_rn(f[1], s), __fmul_rn(f[2], s), __fmul_rn(f[3], s));
+}
+
+// 6-bit symmetric codes: one thread per 8 weights (word w of a 64-weight
+// chunk: low-nibble bytes 4w .. 4w + 3, plane bytes 32 + 2w, 33 + 2w).
+__global__ void dequant_w6_kernel(const uint8_t* __restrict__ codes, const __half* __restrict__ scales,
+                                  int K, long long units, float* __restrict__ out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= units) return;
+    const long long upr = K / 8;
+    const long long n = i / upr;
+    const int k0 = (int)(i % upr) * 8;
+    const uint8_t* chunk = codes + n * (K / 64 * 48) + (k0 / 64) * 48;
+    const int w = (k0 % 64) / 8;
+    const float s = __half2float(scales[n * (K / 16) + k0 / 16]);
+    const uint32_t lo = *reinterpret_cast<const uint32_t*>(chunk + 4 * w);
+    const uint32_t hi = (uint32_t)chunk[32 + 2 * w] | ((uint32_t)chunk[33 + 2 * w] << 8);
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int u = (int)(((lo >> (4 * e)) & 15u) | (((hi >> (2 * e)) & 3u) << 4));
+        o[e] = __fmul_rn((float)(u - 32), s);
+    }
+    float4* dst = reinterpret_cast<float4*>(out + n * K + k0);
+    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
 }
 
 // One thread per 32-bit word of a superblock's low nibbles (32 words, 8
@@ -349,17 +394,15 @@ cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st) {
         pack_done_kernel<<<1, 32, 0, st>>>();
         return cudaGetLastError();
     }
-    const int G = a.fmt == kFmtW4G64 ? 64 : 16;
+    const int G = sym_group(a.fmt);
     const long long groups = N * (a.K / G);
     const unsigned grid = (unsigned)((groups + kPackWarps - 1) / kPackWarps);
-    if (a.fmt == kFmtW4G64)
-        qpack_sym_kernel<64, 7><<<grid, kPackWarps * 32, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo,
-                                                                   a.t_hi, static_cast<uint8_t*>(a.codes),
-                                                                   static_cast<uint16_t*>(a.scales));
-    else
-        qpack_sym_kernel<16, 127><<<grid, kPackWarps * 32, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo,
-                                                                     a.t_hi, static_cast<uint8_t*>(a.codes),
-                                                                     static_cast<uint16_t*>(a.scales));
+    auto kern = a.fmt == kFmtW4G64 ? qpack_sym_kernel<64, 7>
+              : a.fmt == kFmtW8G16 ? qpack_sym_kernel<16, 127>
+              : a.fmt == kFmtW8G64 ? qpack_sym_kernel<64, 127>
+                                   : qpack_sym_kernel<16, 31>;
+    kern<<<grid, kPackWarps * 32, 0, st>>>(a.W, a.K, a.N, a.act_sq, a.n_cand, a.t_lo, a.t_hi,
+                                           static_cast<uint8_t*>(a.codes), static_cast<uint16_t*>(a.scales));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t used = (size_t)groups * 2;
@@ -379,10 +422,15 @@ cudaError_t launch_dequant(int fmt, int K, int N, const void* codes, const void*
         const long long words = (long long)N * K / 8;
         dequant_w4_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
             static_cast<const uint32_t*>(codes), static_cast<const __half*>(scales), K, words, out);
-    } else if (fmt == kFmtW8G16) {
+    } else if (is_w8(fmt)) {
         const long long words = (long long)N * K / 4;
-        dequant_w8_kernel<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
+        auto kern = fmt == kFmtW8G16 ? dequant_w8_kernel<16> : dequant_w8_kernel<64>;
+        kern<<<(unsigned)((words + threads - 1) / threads), threads, 0, st>>>(
             static_cast<const uint32_t*>(codes), static_cast<const __half*>(scales), K, words, out);
+    } else if (fmt == kFmtW6G16) {
+        const long long units = (long long)N * K / 8;
+        dequant_w6_kernel<<<(unsigned)((units + threads - 1) / threads), threads, 0, st>>>(
+            static_cast<const uint8_t*>(codes), static_cast<const __half*>(scales), K, units, out);
     } else {
         const long long words = (long long)N * (K / 256) * 32;
         auto kern = fmt == kFmtW4SB32 ? dequant_sb_kernel<4> : fmt == kFmtW5SB32 ? dequant_sb_kernel<5>

@@ -412,6 +412,40 @@ __device__ __forceinline__ void dq_sbw(const uint4 hd, const uint4 c0, const uin
     }
 }
 
+// 32 6-bit symmetric weights (half of a 64-weight chunk: 16 low-nibble bytes
+// c, 8 plane bytes pl; two fp16 scales, one per 16 weights) -> 16 bf16 pairs.
+// Each code byte u = q + 32 (low nibble plus plane bits 4..5 merged as for
+// the wider superblock codes) goes under the fp16 exponent of 1024:
+// (1024 + u) s - 1056 s = q s, exact in fp32, then one rounding to bf16.
+__device__ __forceinline__ void dq_w6(const uint4 c, const uint2 pl, uint32_t sc, uint32_t (&o)[16]) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t pw[2] = {pl.x, pl.y};
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const uint16_t sb = (uint16_t)(g ? sc >> 16 : sc & 0xffffu);
+        const float cf = __fmul_rn(-1056.0f, __half2float(__ushort_as_half(sb)));   // exact
+#pragma unroll
+        for (int ii = 0; ii < 2; ++ii) {
+            const int i = 2 * g + ii;
+            uint32_t hl, hh;
+            sb_high<6>((pw[i >> 1] >> (16 * (i & 1))) & 0xffffu, hl, hh);
+            const uint32_t lo = merge_nib(w[i], hl), hi = merge_nib(w[i] >> 4, hh);   // u of weights 0,2,4,6 / 1,3,5,7
+            const uint32_t e0 = lop_mask_or(lo, 0x00FF00FFu, 0x64006400u);        // weights 0, 4
+            const uint32_t e1 = lop_mask_or(lo >> 8, 0x00FF00FFu, 0x64006400u);   // weights 2, 6
+            const uint32_t d0 = lop_mask_or(hi, 0x00FF00FFu, 0x64006400u);        // weights 1, 5
+            const uint32_t d1 = lop_mask_or(hi >> 8, 0x00FF00FFu, 0x64006400u);   // weights 3, 7
+            const float v0 = fma_h<0>(e0, sb, cf), v4 = fma_h<1>(e0, sb, cf);
+            const float v2 = fma_h<0>(e1, sb, cf), v6 = fma_h<1>(e1, sb, cf);
+            const float v1 = fma_h<0>(d0, sb, cf), v5 = fma_h<1>(d0, sb, cf);
+            const float v3 = fma_h<0>(d1, sb, cf), v7 = fma_h<1>(d1, sb, cf);
+            o[4 * i + 0] = pack_bf16(v0, v1);
+            o[4 * i + 1] = pack_bf16(v2, v3);
+            o[4 * i + 2] = pack_bf16(v4, v5);
+            o[4 * i + 3] = pack_bf16(v6, v7);
+        }
+    }
+}
+
 // ------------------------------------------------------------ work units
 struct Unit { int item, n0, t0, t1; };
 
@@ -463,7 +497,7 @@ struct ScaleCursor {
         const TcItem& it = p->it[u.item];
         const int n = u.n0 + r;
         row = n < it.N ? it.scales + (size_t)n * it.srb : nullptr;
-        groups = FMT == kFmtW4G64 ? it.K / 64 : it.K / 16;
+        groups = it.K / sym_group(FMT);
         t = u.t0;
     }
     __device__ __forceinline__ void start(const TcArgs<MAXI>* prm, int rr, int hh) {
@@ -483,12 +517,12 @@ struct ScaleCursor {
         const uint8_t* a = spare;
         bool in = false;
         if (valid && row) {
-            const int gi = FMT == kFmtW4G64 ? (KS == 128 ? 2 * t + (h >> 1) : 4 * t + h) : 8 * t + 2 * h;
+            const int gi = sym_group(FMT) == 64 ? (KS == 128 ? 2 * t + (h >> 1) : 4 * t + h) : 8 * t + 2 * h;
             in = gi < groups;
             if (in) a = row + 2 * gi;
         }
         if (is_sb(FMT)) v = 0u;                           // scales travel inside the records
-        else if (FMT == kFmtW4G64) v = ldg_nc_u16(a);
+        else if (sym_group(FMT) == 64) v = ldg_nc_u16(a);
         else v = ldg_nc_u32(a);
         mask = in ? 0xffffffffu : 0u;
         if (valid && ++t >= u.t1) {
@@ -542,7 +576,8 @@ constexpr unsigned kNapCritical = 0, kNapLoader = 64, kNapEpilogue = 512, kNapDr
 
 template <int FMT, int KS, int MAXI>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcArgs<MAXI> p) {
-    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : sb_record(FMT);   // code bytes per row and stage
+    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : is_w8(FMT) ? KS : FMT == kFmtW6G16 ? KS / 64 * 48
+                                                                   : sb_record(FMT);   // code bytes per row and stage
     const int AS = p.AS;                                     // A slots (KS / 2 columns each)
     constexpr uint32_t ACOLS = KS / 2;
     constexpr uint32_t QCOLS = ACOLS / 4;                    // columns one dequantizing thread writes per stage
@@ -685,6 +720,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         const uint32_t cph = code_pos<RB>(r, 0);               // superblock record header
         // high-bit plane of groups 2h, 2h + 1: 8 bytes (5 bits) or 16 (6 bits) at 144 + 8h or 144 + 16h
         const uint32_t cpp = code_pos<RB>(r, 0) + 144u + (FMT == kFmtW6SB32 ? 16u : 8u) * (uint32_t)h;
+        // 6-bit symmetric: quarter h is half h & 1 of 48-byte chunk h >> 1 (16 nibble bytes, 8 plane bytes)
+        const uint32_t cw6 = code_pos<RB>(r, 3 * (h >> 1) + (h & 1));
+        const uint32_t cp6 = code_pos<RB>(r, 3 * (h >> 1) + 2) + 8u * (uint32_t)(h & 1);
         uint32_t g = 0;
         int slot = 0, wrap = 0, aslot = 0, awrap = 0;
         bool ok = true;
@@ -736,12 +774,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     uint32_t o[16];
                     dq_w4<4>(wv, (uint16_t)s, o);
                     tmem_st16(ta, o);
-                } else {                                      // 32 weights: chunks 2h, 2h+1, two groups
+                } else if (FMT == kFmtW6G16) {               // 32 weights: two groups of 16
+                    const uint4 c0 = *reinterpret_cast<const uint4*>(cs + cw6);
+                    const uint2 pl = *reinterpret_cast<const uint2*>(cs + cp6);
+                    uint32_t o[16];
+                    dq_w6(c0, pl, s, o);
+                    tmem_st16(ta, o);
+                } else {                                      // int8, 32 weights: chunks 2h, 2h+1
                     uint4 c[2];
                     c[0] = *reinterpret_cast<const uint4*>(cs + cp0);
                     c[1] = *reinterpret_cast<const uint4*>(cs + cp1);
                     uint32_t o[16];
-                    dq_w8(c, s, o);
+                    dq_w8(c, FMT == kFmtW8G64 ? s * 0x10001u : s, o);   // g64: one scale for both halves
                     tmem_st16(ta, o);
                 }
                 tmem_st_wait();
@@ -872,7 +916,8 @@ bool encode(EncodeTiled enc, CUtensorMap* m, CUtensorMapDataType dt, int rank, c
 
 template <int FMT, int KS, int MAXI>
 cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
-    constexpr uint32_t RB = FMT == kFmtW4G64 ? KS / 2 : FMT == kFmtW8G16 ? KS : sb_record(FMT);
+    constexpr uint32_t RB = FMT == kFmtW4G64 ? KS / 2 : is_w8(FMT) ? KS : FMT == kFmtW6G16 ? KS / 64 * 48
+                                                                        : sb_record(FMT);
     const EncodeTiled enc = encoder();
     if (!enc) return cudaErrorNotSupported;
     TcArgs<MAXI> p = {};
@@ -1006,16 +1051,18 @@ cudaError_t launch_chunks(const WgemmArgs* a, int count, cudaStream_t st) {
 
 }  // namespace
 
-// The 5- and 6-bit superblock formats have no register-path kernel: their
-// products run here at every M (x rows past M are zero-filled by the copy).
+// The 5- and 6-bit formats have no register-path kernel: their products run
+// here at every M (x rows past M are zero-filled by the copy).
 bool tc_supported(int fmt, int M) {
-    if (fmt == kFmtW5SB32 || fmt == kFmtW6SB32) return M >= 1;
-    return M >= kTcMinM && (fmt == kFmtW4G64 || fmt == kFmtW8G16 || fmt == kFmtW4SB32);
+    if (fmt == kFmtW5SB32 || fmt == kFmtW6SB32 || fmt == kFmtW6G16) return M >= 1;
+    return M >= kTcMinM && (fmt == kFmtW4G64 || is_w8(fmt) || fmt == kFmtW4SB32);
 }
 
 cudaError_t launch_tc(const WgemmArgs* a, int count, cudaStream_t st) {
     if (a[0].fmt == kFmtW4G64) return launch_chunks<kFmtW4G64>(a, count, st);
     if (a[0].fmt == kFmtW8G16) return launch_chunks<kFmtW8G16>(a, count, st);
+    if (a[0].fmt == kFmtW8G64) return launch_chunks<kFmtW8G64>(a, count, st);
+    if (a[0].fmt == kFmtW6G16) return launch_chunks<kFmtW6G16>(a, count, st);
     if (a[0].fmt == kFmtW4SB32) return launch_chunks<kFmtW4SB32>(a, count, st);
     if (a[0].fmt == kFmtW5SB32) return launch_chunks<kFmtW5SB32>(a, count, st);
     return launch_chunks<kFmtW6SB32>(a, count, st);

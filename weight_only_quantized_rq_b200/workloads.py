@@ -30,7 +30,7 @@ class Matrix:
     name: str
     K: int          # input features (reduction dim)
     N: int          # output features
-    fmt: str        # "w4g64" | "w8g16" | "w4sb32"
+    fmt: str        # "w4g64" | "w8g16" | "w4sb32" | "w5sb32" | "w6sb32"
     n_cand: int     # 1 = RTN, 64 = E[x^2]-weighted search
     outliers: bool = False
 
@@ -80,6 +80,18 @@ WORKLOADS = [
                 Matrix("ffn_value", 16384, 4096, "w4g64", 64),
                 Matrix("head", 4096, 65536, "w8g16", 64)),
              1, (1, 32, 64, 128), {4096: "eight99"}),
+]
+
+# The COMPRESSION preset's wider codes at 2.9B width (rwkv-quant article, "Two
+# presets and six sizes": ffn.key and head in 5 bits; "Where 2.9B breaks": all
+# of o_proj in 6 bits as the alternative to one bf16 matrix).
+VARIANTS = [
+    Workload(5, "w5sb32-aw-2.9B ffn.key 2560->10240 x32 (COMPRESSION)",
+             (Matrix("ffn_key", 2560, 10240, "w5sb32", 64),), 32, (1, 16), {2560: "eight98"}),
+    Workload(6, "w5sb32-aw-2.9B head 2560->65536 (COMPRESSION)",
+             (Matrix("head", 2560, 65536, "w5sb32", 64),), 1, (1, 16), {2560: "eight98"}),
+    Workload(7, "w6sb32-aw-2.9B o 2560^2 x32 (all of o_proj in 6 bits)",
+             (Matrix("o", 2560, 2560, "w6sb32", 64),), 32, (1, 16), {2560: "eight98"}),
 ]
 
 

@@ -30,7 +30,7 @@ class Matrix:
     name: str
     K: int          # input features (reduction dim)
     N: int          # output features
-    fmt: str        # "w4g64" | "w8g16" | "w4sb32" | "w5sb32" | "w6sb32"
+    fmt: str        # "w4g64" | "w8g16" | "w8g64" | "w6g16" | "w4sb32" | "w5sb32" | "w6sb32"
     n_cand: int     # 1 = RTN, 64 = E[x^2]-weighted search
     outliers: bool = False
 
@@ -82,9 +82,10 @@ WORKLOADS = [
              1, (1, 32, 64, 128), {4096: "eight99"}),
 ]
 
-# The COMPRESSION preset's wider codes at 2.9B width (rwkv-quant article, "Two
-# presets and six sizes": ffn.key and head in 5 bits; "Where 2.9B breaks": all
-# of o_proj in 6 bits as the alternative to one bf16 matrix).
+# Preset variants: the COMPRESSION preset's wider codes at 2.9B width
+# (rwkv-quant article, "Two presets and six sizes": ffn.key and head in 5 bits;
+# "Where 2.9B breaks": all of o_proj in 6 bits as the alternative to one bf16
+# matrix), the REDUCTION preset's 6-bit channel-mix, and the int8 g64 tier.
 VARIANTS = [
     Workload(5, "w5sb32-aw-2.9B ffn.key 2560->10240 x32 (COMPRESSION)",
              (Matrix("ffn_key", 2560, 10240, "w5sb32", 64),), 32, (1, 16), {2560: "eight98"}),
@@ -92,6 +93,15 @@ VARIANTS = [
              (Matrix("head", 2560, 65536, "w5sb32", 64),), 1, (1, 16), {2560: "eight98"}),
     Workload(7, "w6sb32-aw-2.9B o 2560^2 x32 (all of o_proj in 6 bits)",
              (Matrix("o", 2560, 2560, "w6sb32", 64),), 32, (1, 16), {2560: "eight98"}),
+    # the REDUCTION preset's channel-mix in 6 bits (symmetric, group 16)
+    Workload(8, "w6g16-aw-1.5B cmix 2048->8192->2048 x24 (REDUCTION)",
+             (Matrix("ffn_key", 2048, 8192, "w6g16", 64), Matrix("ffn_value", 8192, 2048, "w6g16", 64)),
+             24, (1, 16), {2048: "ch1202x50"}),
+    # the model card's int8 w8g64 tier ("Accuracy warning") on the 1.5B layer set
+    Workload(9, "w8g64-aw-1.5B-layerset x24 (int8 tier)",
+             tuple(Matrix(n, 2048, 2048, "w8g64", 64) for n in "rkvo")
+             + (Matrix("ffn_key", 2048, 8192, "w8g64", 64), Matrix("ffn_value", 8192, 2048, "w8g64", 64)),
+             24, (1, 4, 16), {2048: "ch1202x50"}),
 ]
 
 

@@ -84,6 +84,10 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_act_sumsq.restype = None
     L.orc_act_finalize.argtypes = [_P, _i, ctypes.c_longlong, _P]
     L.orc_act_finalize.restype = None
+    L.orc_hessian_accum.argtypes = [_P, _i, _i, _P]
+    L.orc_hessian_accum.restype = None
+    L.orc_gptq_pack_sym.argtypes = [_P, _i, _i, _P, _P, _P, _i, _i, _f, _f, _P, _P]
+    L.orc_gptq_pack_sym.restype = None
     L.orc_threads.argtypes = []
     L.orc_threads.restype = _i
     L.orc_set_threads.argtypes = [_i]
@@ -275,3 +279,53 @@ def act_finalize(sum_sq, rows: int) -> np.ndarray:
     out = np.zeros(s.size, dtype=np.float32)
     lib().orc_act_finalize(_ptr(s), s.size, int(rows), _ptr(out))
     return out
+
+
+# --------------------------------------------------------------------- GPTQ --
+def hessian_accum(x_bf16_bits, H=None) -> np.ndarray:
+    """H += x^T x (fp64 [K][K]) over the bf16 rows x [R][K], every element
+    summed in ascending row order."""
+    x = _c(x_bf16_bits, np.uint16)
+    R, K = x.shape
+    out = np.zeros((K, K), np.float64) if H is None else _c(H, np.float64).copy()
+    lib().orc_hessian_accum(_ptr(x), R, K, _ptr(out))
+    return out
+
+
+def gptq_prepare(H, damp: float = 0.01):
+    """The factor GPTQ's column loop needs (Frantar et al. 2022): columns with
+    H_kk == 0 are dead (H_kk := 1, their weights are zeroed); the diagonal is
+    damped by damp * mean(diag H); U = the upper Cholesky factor of H^-1,
+    computed as in the method's description: Cholesky of H, the inverse from
+    it, Cholesky of the inverse. numpy's LAPACK routines are the library
+    steps. Returns (U fp64 [K][K] upper, dead uint8 [K])."""
+    H = np.array(H, dtype=np.float64, copy=True)
+    K = H.shape[0]
+    d = np.diag(H).copy()
+    dead = d == 0.0
+    H[np.arange(K)[dead], np.arange(K)[dead]] = 1.0
+    lam = damp * np.mean(np.diag(H))
+    H[np.arange(K), np.arange(K)] += lam
+    L = np.linalg.cholesky(H)
+    Linv = np.linalg.inv(L)
+    Hinv = Linv.T @ Linv
+    U = np.linalg.cholesky(Hinv).T
+    return np.ascontiguousarray(np.triu(U)), dead.astype(np.uint8)
+
+
+def gptq_pack(fmt: str, W, U, dead, act_sq=None, n_cand: int = 64, t_lo: float = 0.7, t_hi: float = 1.0):
+    """GPTQ on the preset's grid for a symmetric format; the same planes as
+    pack(). Returns (codes, scales)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    U = _c(U, np.float64)
+    dead = _c(dead, np.uint8)
+    a = None if act_sq is None else _c(act_sq, np.float32)
+    cshape, cdt, sshape = packed_shapes(fmt, K, N)
+    if sshape is None:
+        raise ValueError("GPTQ is built for the symmetric formats")
+    codes = np.zeros(cshape, dtype=cdt)
+    scales = np.zeros(sshape, dtype=np.uint16)
+    lib().orc_gptq_pack_sym(_ptr(W), K, N, _ptr(U), _ptr(dead), _ptr(a), FORMATS[fmt], n_cand, t_lo, t_hi,
+                            _ptr(codes), _ptr(scales))
+    return codes, scales

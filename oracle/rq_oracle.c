@@ -232,6 +232,30 @@ int orc_sym_group(const float *w, const float *a, int G, int qmax,
  *                  scales [N][K/16] fp16. 7 bits per weight. The layout is
  *                  this project's own (the pages give only the bit width).
  * a == NULL means every a_k = 1 (plain MSE search). */
+/* Write the codes of row n (qrow[k], k = 0..K-1) in the format's layout. */
+static void emit_sym_row(uint8_t *codes, int bits, int K, int n, const int8_t *qrow)
+{
+    for (size_t kk = 0; kk < (size_t)K; kk++) {
+        int qk = qrow[kk];
+        if (bits == 8) {
+            codes[(size_t)n * K + kk] = (uint8_t)(qk + 128);
+        } else if (bits == 6) {
+            int u = qk + 32;
+            uint8_t *chunk = codes + (size_t)n * (K / 64 * 48) + (kk / 64) * 48;
+            size_t j = kk % 64;
+            if ((j & 1) == 0) chunk[j / 2] = (uint8_t)(u & 15);
+            else chunk[j / 2] = (uint8_t)(chunk[j / 2] | ((u & 15) << 4));
+            if (j % 4 == 0) chunk[32 + j / 4] = 0;
+            chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (2 * (j % 4)));
+        } else {
+            uint8_t u = (uint8_t)(qk + 8);
+            uint8_t *byte = codes + (size_t)n * (K / 2) + kk / 2;
+            if ((kk & 1) == 0) *byte = u;
+            else *byte = (uint8_t)(*byte | (u << 4));
+        }
+    }
+}
+
 void orc_pack_sym(const float *W, int K, int N, const float *a, int fmt,
                   int n_cand, float t_lo, float t_hi, uint8_t *codes, uint16_t *scales)
 {
@@ -243,33 +267,98 @@ void orc_pack_sym(const float *W, int K, int N, const float *a, int fmt,
     orc_grid(n_cand, t_lo, t_hi, t);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int n = 0; n < N; n++) {
-        int8_t q[64];
+        int8_t *qrow = (int8_t *)malloc((size_t)K);
         const float *row = W + (size_t)n * K;
         for (int g = 0; g < ng; g++) {
             uint16_t s;
             orc_sym_group(row + (size_t)g * G, a ? a + (size_t)g * G : NULL, G, qmax,
-                          t, n_cand, &s, q, NULL);
+                          t, n_cand, &s, qrow + (size_t)g * G, NULL);
             scales[(size_t)n * ng + g] = s;
-            for (int k = 0; k < G; k++) {
-                size_t kk = (size_t)g * G + k;
-                if (bits == 8) {
-                    codes[(size_t)n * K + kk] = (uint8_t)(q[k] + 128);
-                } else if (bits == 6) {
-                    int u = q[k] + 32;
-                    uint8_t *chunk = codes + (size_t)n * (K / 64 * 48) + (kk / 64) * 48;
-                    size_t j = kk % 64;
-                    if ((j & 1) == 0) chunk[j / 2] = (uint8_t)(u & 15);
-                    else chunk[j / 2] = (uint8_t)(chunk[j / 2] | ((u & 15) << 4));
-                    if (j % 4 == 0) chunk[32 + j / 4] = 0;
-                    chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (2 * (j % 4)));
-                } else {
-                    uint8_t u = (uint8_t)(q[k] + 8);
-                    uint8_t *byte = codes + (size_t)n * (K / 2) + kk / 2;
-                    if ((kk & 1) == 0) *byte = u;
-                    else *byte = (uint8_t)(*byte | (u << 4));
-                }
+        }
+        emit_sym_row(codes, bits, K, n, qrow);
+        free(qrow);
+    }
+    free(t);
+}
+
+/* ------------------------------------------------------------------------ */
+/* GPTQ on the preset's grid (symmetric formats)                            */
+/* ------------------------------------------------------------------------ */
+
+/* Running Hessian of the layer's input: H[i][j] += sum_r x[r][i] * x[r][j]
+ * over the R bf16 rows of this call (row-major [R][K]), every element summed
+ * in fp64 in ascending r starting from 0, then added to H. Products of two
+ * bf16 values are exact in fp64. GPTQ's factor 2/R scales H uniformly and
+ * changes nothing below (the damping is relative), so it is left out. */
+void orc_hessian_accum(const uint16_t *x, int R, int K, double *H)
+{
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < K; i++) {
+        for (int j = 0; j < K; j++) {
+            double acc = 0.0;
+            for (int r = 0; r < R; r++) {
+                double xi = (double)orc_bf16_to_f32(x[(size_t)r * K + i]);
+                double xj = (double)orc_bf16_to_f32(x[(size_t)r * K + j]);
+                acc = acc + xi * xj;
+            }
+            H[(size_t)i * K + j] = H[(size_t)i * K + j] + acc;
+        }
+    }
+}
+
+/* GPTQ (Frantar et al., "GPTQ: Accurate Post-Training Quantization for
+ * Generative Pre-trained Transformers", 2022), restated for the preset's
+ * symmetric formats; [ART] "Calibration leakage and honest measurements": GPTQ
+ * on the preset's grid without changing the format, the kernels or the file size;
+ * [CARD]: symmetric int4 group 64, GPTQ-calibrated.
+ *   U       fp64 [K][K], the upper Cholesky factor of the damped inverse
+ *           Hessian (H^-1 = U^T U; only the upper triangle is read)
+ *   dead    [K], 1 where the Hessian's diagonal was 0: those columns of W
+ *           are set to 0 before quantization
+ * Per row, columns k = 0..K-1 in order, w the row in fp64:
+ *   at the first column of each group: the group's scale is the preset's
+ *   E[x^2]-weighted search (orc_sym_group) on fp32(w) of the group's current
+ *   weights;
+ *   q_k = clamp(rint(fp32(w_k) / s), -qmax, qmax);
+ *   err = (w_k - q_k s) / U[k][k];  w_j = w_j - err * U[k][j] for j > k
+ *   (fp64, one rounding per operation, the updates of w_j in ascending k).
+ * The codes and scales land in the same planes as orc_pack_sym's. */
+void orc_gptq_pack_sym(const float *W, int K, int N, const double *U, const uint8_t *dead,
+                       const float *a, int fmt, int n_cand, float t_lo, float t_hi,
+                       uint8_t *codes, uint16_t *scales)
+{
+    int bits = sym_bits(fmt);
+    int G = sym_gsize(fmt);
+    int qmax = (1 << (bits - 1)) - 1;
+    int ng = K / G;
+    float *t = (float *)malloc(sizeof(float) * (size_t)n_cand);
+    orc_grid(n_cand, t_lo, t_hi, t);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < N; n++) {
+        double *w = (double *)malloc(sizeof(double) * (size_t)K);
+        int8_t *qrow = (int8_t *)malloc((size_t)K);
+        for (int k = 0; k < K; k++) w[k] = dead[k] ? 0.0 : (double)W[(size_t)n * K + k];
+        for (int g = 0; g < ng; g++) {
+            int k0 = g * G;
+            float wg[64];
+            int8_t qg[64];
+            uint16_t s;
+            for (int i = 0; i < G; i++) wg[i] = (float)w[k0 + i];
+            orc_sym_group(wg, a ? a + k0 : NULL, G, qmax, t, n_cand, &s, qg, NULL);
+            scales[(size_t)n * ng + g] = s;
+            float sf = orc_f16_to_f32(s);
+            for (int i = 0; i < G; i++) {
+                int k = k0 + i;
+                int q = sym_code((float)w[k], sf, qmax);
+                qrow[k] = (int8_t)q;
+                double d = w[k] - (double)((float)q * sf);
+                double err = d / U[(size_t)k * K + k];
+                for (int j = k + 1; j < K; j++) w[j] = w[j] - err * U[(size_t)k * K + j];
             }
         }
+        emit_sym_row(codes, bits, K, n, qrow);
+        free(w);
+        free(qrow);
     }
     free(t);
 }

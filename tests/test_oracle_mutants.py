@@ -17,8 +17,8 @@ MUTANTS = [
     ("drop the E[x^2] weight", "L = L + ak * e;", "L = L + e;", None),
     ("ties go to the last index", "L < bestL", "L <= bestL", None),
     ("qmax = 2^(b-1)", "int qmax = (1 << (bits - 1)) - 1;", "int qmax = (1 << (bits - 1));", None),
-    ("nibbles swapped", "if ((kk & 1) == 0) *byte = u;\n                    else *byte = (uint8_t)(*byte | (u << 4));",
-     "if ((kk & 1) == 1) *byte = u;\n                    else *byte = (uint8_t)(*byte | (u << 4));", None),
+    ("nibbles swapped", "if ((kk & 1) == 0) *byte = u;\n            else *byte = (uint8_t)(*byte | (u << 4));",
+     "if ((kk & 1) == 1) *byte = u;\n            else *byte = (uint8_t)(*byte | (u << 4));", None),
     ("search on the unrounded scale", "float sf = orc_f16_to_f32(sh);\n        double L", "float sf = prod;\n        double L", None),
     ("truncate instead of rint", "float r = rintf(clampf(v, -(float)qmax, (float)qmax));",
      "float r = truncf(clampf(v, -(float)qmax, (float)qmax));", None),
@@ -31,19 +31,26 @@ MUTANTS = [
     ("grid misses its top end", "step = step / (double)(n - 1);", "step = step / (double)n;", None),
     ("superblock min from the scales", "if (M_star[j] > mM) mM = M_star[j];", "if (S_star[j] > mM) mM = S_star[j];", None),
     ("product sums the wrong row of x", "const double *xm = xd + (size_t)m * K;", "const double *xm = xd;", None),
-    ("int8 code offset 127", "codes[(size_t)n * K + kk] = (uint8_t)(q[k] + 128);",
-     "codes[(size_t)n * K + kk] = (uint8_t)(q[k] + 127);", None),
+    ("int8 code offset 127", "codes[(size_t)n * K + kk] = (uint8_t)(qk + 128);",
+     "codes[(size_t)n * K + kk] = (uint8_t)(qk + 127);", None),
     ("dequant drops the group index", "float s = orc_f16_to_f32(scales[(size_t)n * ng + k / G]);",
      "float s = orc_f16_to_f32(scales[(size_t)n * ng]);", None),
     ("sb dequant adds the min", "float p = (float)q * S;\n    return p - M;", "float p = (float)q * S;\n    return p + M;", None),
     ("absmax from the last element", "if (v > absmax) absmax = v;", "absmax = v;", None),
     ("6-bit symmetric plane bit order", "chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (2 * (j % 4)));",
      "chunk[32 + j / 4] |= (uint8_t)((u >> 4) << (6 - 2 * (j % 4)));", None),
-    ("6-bit symmetric code offset 31", "int u = q[k] + 32;", "int u = q[k] + 31;", None),
+    ("6-bit symmetric code offset 31", "int u = qk + 32;", "int u = qk + 31;", None),
     ("6-bit symmetric low nibbles swapped", "if ((j & 1) == 0) chunk[j / 2] = (uint8_t)(u & 15);",
      "if ((j & 1) == 1) chunk[j / 2] = (uint8_t)(u & 15);", None),
     ("int8 g64 search on the first 16 weights", "orc_sym_group(row + (size_t)g * G, a ? a + (size_t)g * G : NULL, G, qmax,",
      "orc_sym_group(row + (size_t)g * G, a ? a + (size_t)g * G : NULL, G == 64 && bits == 8 ? 16 : G, qmax,", None),
+    ("GPTQ update adds the error", "w[j] = w[j] - err * U[(size_t)k * K + j];", "w[j] = w[j] + err * U[(size_t)k * K + j];", None),
+    ("GPTQ divides by the wrong diagonal", "double err = d / U[(size_t)k * K + k];", "double err = d / U[(size_t)k0 * K + k0];", None),
+    ("GPTQ scale from the original weights", "for (int i = 0; i < G; i++) wg[i] = (float)w[k0 + i];",
+     "for (int i = 0; i < G; i++) wg[i] = W[(size_t)n * K + k0 + i];", None),
+    ("GPTQ keeps dead columns", "w[k] = dead[k] ? 0.0 : (double)W[(size_t)n * K + k];", "w[k] = (double)W[(size_t)n * K + k];", None),
+    ("GPTQ code from the group search's codes", "int q = sym_code((float)w[k], sf, qmax);", "int q = qg[i];", None),
+    ("Hessian skips the last row", "for (int r = 0; r < R; r++) {\n                double xi", "for (int r = 0; r < R - 1; r++) {\n                double xi", None),
     ("E[x^2] sums |x| instead of x^2", "part = part + v * v;", "part = part + fabs(v);", None),
     ("E[x^2] skips the last chunk", "for (int c = 0; c < 64; c++) {\n            int r0", "for (int c = 0; c < 63; c++) {\n            int r0", None),
     ("E[x^2] divides by rows - 1", "act_sq[k] = (float)(sum_sq[k] / (double)rows);", "act_sq[k] = (float)(sum_sq[k] / (double)(rows - 1));", None),

@@ -577,3 +577,111 @@ def test_act_stats_match_numpy_and_accumulate(orc):
     a = orc.act_finalize(s, R)
     assert np.allclose(a, (ref / R).astype(np.float32), rtol=1e-6, atol=0)
     assert int(np.argmax(a)) == 7
+
+
+# ------------------------------------------------------------------ GPTQ ---
+def test_hessian_accum_exact_integers(orc):
+    """Small-integer bf16 rows: every product and sum is an exact integer, so
+    H must equal the integer x^T x, and two calls accumulate."""
+    rng = np.random.default_rng(61)
+    x = rng.integers(-9, 10, size=(37, 24))
+    xb = _bf16_bits(x.astype(np.float32))
+    H = orc.hessian_accum(xb)
+    assert np.array_equal(H, (x.T @ x).astype(np.float64))
+    H2 = orc.hessian_accum(xb[20:], orc.hessian_accum(xb[:20]))
+    assert np.array_equal(H2, H)
+
+
+def _sym_codes_np(w32, sf, qmax):
+    if sf == 0.0:
+        return np.zeros_like(w32, dtype=np.int64)
+    v = (w32 / np.float32(sf)).astype(np.float32)
+    return np.rint(np.clip(v, -qmax, qmax)).astype(np.int64)
+
+
+def _gptq_by_obs(orc, fmt, W, H, a, n_cand, damp=0.01):
+    """GPTQ written a second way: after quantizing column k, the not yet
+    quantized columns F = k+1.. move by the optimal-brain-surgeon update
+    computed from the damped Hessian restricted to {k} u F (an explicit
+    inverse of that block; no Cholesky factor)."""
+    G, qmax = orc.GROUP[fmt], orc.QMAX[fmt]
+    N, K = W.shape
+    Hd = np.array(H, dtype=np.float64, copy=True)
+    dead = np.diag(Hd) == 0
+    Hd[dead, dead] = 1.0
+    Hd[np.arange(K), np.arange(K)] += damp * np.mean(np.diag(Hd))
+    codes = np.zeros((N, K), np.int64)
+    scales = np.zeros((N, K // G), np.uint16)
+    for n in range(N):
+        w = W[n].astype(np.float64)
+        w[dead] = 0.0
+        for g in range(K // G):
+            k0 = g * G
+            _, s, _, _ = orc.sym_group(w[k0:k0 + G].astype(np.float32), None if a is None else a[k0:k0 + G],
+                                       qmax, n_cand)
+            scales[n, g] = s
+            sf = float(orc.f16_bits_to_f32(np.array([s], np.uint16))[0])
+            for k in range(k0, k0 + G):
+                q = int(_sym_codes_np(np.array([w[k]], np.float32), sf, qmax)[0])
+                codes[n, k] = q
+                e = w[k] - float(np.float32(q) * np.float32(sf))
+                Hinv = np.linalg.inv(Hd[k:, k:])
+                w[k:] -= e * Hinv[:, 0] / Hinv[0, 0]
+    return codes, scales
+
+
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g16", "w6g16"])
+def test_gptq_matches_sequential_obs(orc, fmt):
+    rng = np.random.default_rng(67)
+    N, K, R = 3, 128, 400
+    mix = rng.standard_normal((K, K)) * 0.3 + np.eye(K)       # correlated channels
+    x = (rng.standard_normal((R, K)) @ mix).astype(np.float32)
+    xb = _bf16_bits(x)
+    H = orc.hessian_accum(xb)
+    a = (np.diag(H) / R).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    U, dead = orc.gptq_prepare(H)
+    codes, scales = orc.gptq_pack(fmt, W, U, dead, a, n_cand=16)
+    q_ref, s_ref = _gptq_by_obs(orc, fmt, W, H, a, 16)
+    assert np.array_equal(scales, s_ref)
+    wd = orc.dequant(fmt, K, N, codes, scales).astype(np.float64)
+    sf = orc.f16_bits_to_f32(s_ref).reshape(N, -1).astype(np.float64).repeat(orc.GROUP[fmt], axis=1)
+    assert np.array_equal(wd, q_ref * sf)
+
+
+@pytest.mark.parametrize("fmt", ["w4g64", "w8g64"])
+def test_gptq_diagonal_hessian_is_the_preset_pack(orc, fmt):
+    """Uncorrelated channels (diagonal H): U is diagonal, no column moves, and
+    GPTQ gives the preset pack's bytes; a dead channel's weights become 0."""
+    rng = np.random.default_rng(71)
+    N, K = 5, 256
+    d = rng.random(K) * 3 + 0.5
+    d[7] = 0.0                                               # a channel that never fires
+    H = np.diag(d)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    a = rng.random(K).astype(np.float32) + 0.1
+    U, dead = orc.gptq_prepare(H)
+    assert np.count_nonzero(np.triu(U, 1)) == 0 and dead[7] == 1 and dead.sum() == 1
+    c1, s1 = orc.gptq_pack(fmt, W, U, dead, a, n_cand=32)
+    W0 = W.copy()
+    W0[:, 7] = 0.0
+    c0, s0 = orc.pack(fmt, W0, a, n_cand=32)
+    assert np.array_equal(c1, c0) and np.array_equal(s1, s0)
+
+
+def test_gptq_lowers_the_output_error(orc):
+    """On strongly correlated inputs GPTQ's output error
+    tr((W - W_hat) H (W - W_hat)^T) is well below the per-group search's."""
+    rng = np.random.default_rng(73)
+    N, K, R = 16, 256, 600
+    basis = rng.standard_normal((24, K))
+    x = (rng.standard_normal((R, 24)) @ basis + 0.05 * rng.standard_normal((R, K))).astype(np.float32)
+    H = orc.hessian_accum(_bf16_bits(x))
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    U, dead = orc.gptq_prepare(H)
+    cg, sg = orc.gptq_pack("w4g64", W, U, dead, None, n_cand=1)
+    cr, sr = orc.pack("w4g64", W, None, n_cand=1)
+    def out_err(c, s):
+        D = W.astype(np.float64) - orc.dequant("w4g64", K, N, c, s).astype(np.float64)
+        return float(np.einsum("nk,kl,nl->", D, H, D))
+    assert out_err(cg, sg) < 0.7 * out_err(cr, sr)

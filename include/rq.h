@@ -52,7 +52,8 @@ typedef enum rq_status {
     RQ_ERR_FORMAT_MISMATCH = 3,    /* descriptor's fmt/K/N differ from the call's */
     RQ_ERR_MISALIGNED = 4,         /* a device pointer is not 16-byte aligned */
     RQ_ERR_CUDA = 5,               /* a CUDA runtime call failed */
-    RQ_ERR_DEVICE_TIMEOUT = 6      /* a bounded device wait gave up (see rq_device_status) */
+    RQ_ERR_DEVICE_TIMEOUT = 6,     /* a bounded device wait gave up (see rq_device_status) */
+    RQ_ERR_NOT_POSITIVE_DEFINITE = 7  /* a GPTQ factorization met a non-positive pivot (rq_device_status) */
 } rq_status;
 
 /* Packed formats.
@@ -237,6 +238,46 @@ int rq_act_sumsq(const void *x, int R, int K, double *sum_sq, void *stream);
  *   rows    total calibration rows summed, >= 1. */
 int rq_act_finalize(const double *sum_sq, int K, long long rows, float *act_sq, void *stream);
 
+/* GPTQ on the preset's grid ([ART] "Calibration leakage and honest
+ * measurements": GPTQ on the preset's grid without changing the format, the
+ * kernels or the file size; [CARD]: symmetric int4 group 64, GPTQ-calibrated).
+ * The method is GPTQ (Frantar et al., 2022), in three calls:
+ *
+ * rq_hessian_accum: H += x^T x for the layer's calibration inputs.
+ *   x  device bf16 [R][K] (raw bits), H device fp64 [K][K], caller-owned,
+ *   zeroed before the first batch. Each element is summed in fp64 in
+ *   ascending row order from 0 and then added to H (products of bf16 values
+ *   are exact in fp64, so the result is bit-reproducible). GPTQ's factor
+ *   2/rows is left out: it scales H uniformly and the damping is relative.
+ *   Limits: 1 <= R <= 2^24, 1 <= K <= 32768. */
+int rq_hessian_accum(const void *x, int R, int K, double *H, void *stream);
+
+/* rq_gptq_prepare: the factor of the column loop.
+ *   H     device fp64 [K][K] (read only)
+ *   damp  relative damping (GPTQ's usual value: 0.01), finite, >= 0
+ *   U     device fp64 [K][K], out: the upper Cholesky factor of the inverse of
+ *         H' = H with zero diagonal entries set to 1, plus damp * mean(diag)
+ *         on the diagonal (H'^-1 = U^T U; zeros below the diagonal). U is the
+ *         workspace too; it must not overlap H.
+ *   dead  device [K] bytes, out: 1 where H's diagonal entry was 0.
+ * Computed as J inv(chol(J H' J)) J (J reverses the index order): one
+ * Cholesky and one triangular inverse, one launch per column (K launches).
+ * A non-positive pivot sets bit 5 of the device status word (see
+ * rq_device_status) and leaves NaNs in U. Limits: 1 <= K <= 16384. */
+int rq_gptq_prepare(const double *H, int K, double damp, double *U, unsigned char *dead, void *stream);
+
+/* rq_gptq_quantize_pack: quantize W into `out` (a symmetric format:
+ * RQ_W4_SYM_G64, RQ_W8_SYM_G16, RQ_W8_SYM_G64 or RQ_W6_SYM_G16; the same
+ * planes as rq_quantize_pack). Per row, in fp64, columns in order: dead
+ * columns start at 0; at each group's first column the group's scale is
+ * rq_quantize_pack's search (act_sq, search as there) on the group's current
+ * weights rounded to fp32; then q_k = clamp(rint(fp32(w_k) / s), +-qmax),
+ * err = (w_k - q_k s) / U[k][k] and w_j -= err * U[k][j] for j > k.
+ *   W device fp32 [N][K]; U, dead from rq_gptq_prepare. K <= 16384.
+ * Same ordering rules as rq_quantize_pack. */
+int rq_gptq_quantize_pack(const float *W, int K, int N, const double *U, const unsigned char *dead,
+                          const float *act_sq, const rq_search *search, const rq_packed *out, void *stream);
+
 /* Static description of a status code. Never NULL. */
 const char *rq_status_string(int status);
 
@@ -244,9 +285,11 @@ const char *rq_status_string(int status);
 int rq_last_cuda_error(void);
 
 /* Reads and clears the device status word that bounded waits inside the
- * tensor-core kernels set when they give up. Synchronizes `stream`.
- * Writes the word to *word (0 = no timeout since the last read) and returns
- * RQ_OK, RQ_ERR_DEVICE_TIMEOUT if the word was non-zero, or RQ_ERR_CUDA. */
+ * kernels set when they give up, and that rq_gptq_prepare sets for a
+ * non-positive pivot (bit 5). Synchronizes `stream`. Writes the word to *word
+ * (0 = nothing since the last read) and returns RQ_OK,
+ * RQ_ERR_DEVICE_TIMEOUT if a wait bit was set, RQ_ERR_NOT_POSITIVE_DEFINITE
+ * if only the pivot bit was, or RQ_ERR_CUDA. */
 int rq_device_status(void *stream, int *word);
 
 /* Library version, major * 10000 + minor * 100 + patch. */

@@ -122,6 +122,30 @@ def test_quantize_pack_validation(L):
     assert L.rq_quantize_pack(A, 4096, 64, None, None, ctypes.byref(d), st) == rq.RQ_ERR_FORMAT_MISMATCH
 
 
+def test_gptq_validation(L):
+    st = ctypes.c_void_p(0)
+    B = ctypes.c_void_p(0x80000)        # a second aligned fake device address
+    assert L.rq_hessian_accum(None, 8, 64, A, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_hessian_accum(A, 0, 64, B, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_hessian_accum(A, 8, 32769, B, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_hessian_accum(U, 8, 64, B, st) == rq.RQ_ERR_MISALIGNED
+    assert L.rq_gptq_prepare(A, 64, 0.01, None, B, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_gptq_prepare(A, 16385, 0.01, B, B, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_gptq_prepare(A, 64, -1.0, B, B, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_gptq_prepare(A, 64, float("nan"), B, B, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_gptq_prepare(A, 64, 0.01, A, B, st) == rq.RQ_ERR_INVALID_ARG       # U overlaps H
+    assert L.rq_gptq_prepare(U, 64, 0.01, B, B, st) == rq.RQ_ERR_MISALIGNED
+    d = _desc("w4g64", 2048, 64)
+    assert L.rq_gptq_quantize_pack(A, 2048, 64, None, B, None, None, ctypes.byref(d), st) == rq.RQ_ERR_INVALID_ARG
+    sb = _desc("w4sb32", 2048, 64, scales=0)
+    assert L.rq_gptq_quantize_pack(A, 2048, 64, B, B, None, None, ctypes.byref(sb), st) == rq.RQ_ERR_INVALID_ARG
+    wide = _desc("w4g64", 32768, 4)
+    assert L.rq_gptq_quantize_pack(A, 32768, 4, B, B, None, None, ctypes.byref(wide), st) == rq.RQ_ERR_UNSUPPORTED_SHAPE
+    assert L.rq_gptq_quantize_pack(A, 1024, 64, B, B, None, None, ctypes.byref(d), st) == rq.RQ_ERR_FORMAT_MISMATCH
+    assert L.rq_gptq_quantize_pack(U, 2048, 64, B, B, None, None, ctypes.byref(d), st) == rq.RQ_ERR_MISALIGNED
+    assert rq.rq_status_string(rq.RQ_ERR_NOT_POSITIVE_DEFINITE) != "unknown status"
+
+
 def test_dequant_validation(L):
     st = ctypes.c_void_p(0)
     d = _desc("w4sb32", 512, 8, scales=0)

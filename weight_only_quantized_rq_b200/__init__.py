@@ -31,6 +31,7 @@ RQ_ERR_FORMAT_MISMATCH = 3
 RQ_ERR_MISALIGNED = 4
 RQ_ERR_CUDA = 5
 RQ_ERR_DEVICE_TIMEOUT = 6
+RQ_ERR_NOT_POSITIVE_DEFINITE = 7
 
 RQ_W4_SYM_G64 = 1
 RQ_W8_SYM_G16 = 2
@@ -44,7 +45,7 @@ FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_AS
               "w6g16": RQ_W6_SYM_G16}
 SB_FORMATS = (RQ_W4_ASYM_SB32, RQ_W5_ASYM_SB32, RQ_W6_ASYM_SB32)
 EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_dequant",
-           "rq_act_sumsq", "rq_act_finalize",
+           "rq_act_sumsq", "rq_act_finalize", "rq_hessian_accum", "rq_gptq_prepare", "rq_gptq_quantize_pack",
            "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
 MAX_BATCH = 160
 TC_MIN_M = 3         # activation rows from which int4/int8/4-bit superblock products run on the tensor cores
@@ -110,6 +111,12 @@ def _lib() -> ctypes.CDLL:
         L.rq_act_sumsq.restype = I
         L.rq_act_finalize.argtypes = [P, I, ctypes.c_longlong, P, P]
         L.rq_act_finalize.restype = I
+        L.rq_hessian_accum.argtypes = [P, I, I, P, P]
+        L.rq_hessian_accum.restype = I
+        L.rq_gptq_prepare.argtypes = [P, I, ctypes.c_double, P, P, P]
+        L.rq_gptq_prepare.restype = I
+        L.rq_gptq_quantize_pack.argtypes = [P, I, I, P, P, P, ctypes.POINTER(RqSearch), ctypes.POINTER(RqPacked), P]
+        L.rq_gptq_quantize_pack.restype = I
         L.rq_status_string.argtypes = [I]
         L.rq_status_string.restype = ctypes.c_char_p
         L.rq_last_cuda_error.argtypes = []
@@ -270,11 +277,52 @@ def rq_act_finalize(sum_sq: torch.Tensor, rows: int, out: torch.Tensor | None = 
     return out
 
 
+def rq_hessian_accum(x: torch.Tensor, H: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H += x^T x (x bf16 [R][K] on the GPU; H fp64 [K][K], created as zeros
+    when None), each element summed in ascending row order. Returns H."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 [R][K] tensor")
+    R, K = int(x.shape[0]), int(x.shape[1])
+    if H is None:
+        H = torch.zeros(K, K, dtype=torch.float64, device=x.device)
+    _check(_lib().rq_hessian_accum(_ptr(x), R, K, _ptr(H), _stream(stream)), "rq_hessian_accum")
+    return H
+
+
+def rq_gptq_prepare(H: torch.Tensor, damp: float = 0.01, U: torch.Tensor | None = None,
+                    dead: torch.Tensor | None = None, stream=None):
+    """The upper Cholesky factor U of the damped inverse Hessian and the dead
+    channel flags (H fp64 [K][K] on the GPU). Returns (U, dead)."""
+    K = int(H.shape[0])
+    if U is None:
+        U = torch.empty(K, K, dtype=torch.float64, device=H.device)
+    if dead is None:
+        dead = torch.empty(K, dtype=torch.uint8, device=H.device)
+    _check(_lib().rq_gptq_prepare(_ptr(H), K, float(damp), _ptr(U), _ptr(dead), _stream(stream)), "rq_gptq_prepare")
+    return U, dead
+
+
+def rq_gptq_quantize_pack(W: torch.Tensor, fmt, U: torch.Tensor, dead: torch.Tensor,
+                          act_sq: torch.Tensor | None = None, n_cand: int = 64, t_lo: float = 0.7, t_hi: float = 1.0,
+                          out: Packed | None = None, stream=None) -> Packed:
+    """GPTQ on the preset's grid: quantize W (fp32 [N][K], CUDA) into a
+    symmetric format with the factor of rq_gptq_prepare. Returns the Packed
+    matrix (same planes as rq_quantize_pack)."""
+    N, K = W.shape
+    if out is None:
+        out = alloc_packed(fmt, K, N, W.device)
+    sr = RqSearch(int(n_cand), float(t_lo), float(t_hi))
+    d = out.desc()
+    _check(_lib().rq_gptq_quantize_pack(_ptr(W), int(K), int(N), _ptr(U), _ptr(dead), _ptr(act_sq), ctypes.byref(sr),
+                                        ctypes.byref(d), _stream(stream)), "rq_gptq_quantize_pack")
+    return out
+
+
 def rq_device_status(stream=None) -> int:
     """Read and clear the device status word (synchronizes the stream)."""
     word = ctypes.c_int(0)
     st = _lib().rq_device_status(_stream(stream), ctypes.byref(word))
-    if st not in (RQ_OK, RQ_ERR_DEVICE_TIMEOUT):
+    if st not in (RQ_OK, RQ_ERR_DEVICE_TIMEOUT, RQ_ERR_NOT_POSITIVE_DEFINITE):
         raise RqError(st, "rq_device_status")
     return word.value
 

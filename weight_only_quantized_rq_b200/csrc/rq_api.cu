@@ -95,6 +95,43 @@ int rq_quantize_pack(const float* W, int K, int N, const float* act_sq, const rq
     return cuda_status(rq::launch_quantize_pack(a, static_cast<cudaStream_t>(stream)));
 }
 
+int rq_hessian_accum(const void* x, int R, int K, double* H, void* stream) {
+    if (!x || !H) return RQ_ERR_INVALID_ARG;
+    if (R < 1 || R > (1 << 24) || K < 1 || K > 32768) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(H)) return RQ_ERR_MISALIGNED;
+    return cuda_status(rq::launch_hessian(x, R, K, H, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_gptq_prepare(const double* H, int K, double damp, double* U, unsigned char* dead, void* stream) {
+    if (!H || !U || !dead) return RQ_ERR_INVALID_ARG;
+    if (K < 1 || K > 16384 || !std::isfinite(damp) || damp < 0.0) return RQ_ERR_INVALID_ARG;
+    const uintptr_t h0 = reinterpret_cast<uintptr_t>(H), u0 = reinterpret_cast<uintptr_t>(U);
+    const uintptr_t bytes = (uintptr_t)K * (uintptr_t)K * sizeof(double);
+    if (h0 < u0 + bytes && u0 < h0 + bytes) return RQ_ERR_INVALID_ARG;      // H and U must not overlap
+    if (!aligned16(H) || !aligned16(U)) return RQ_ERR_MISALIGNED;
+    return cuda_status(rq::launch_gptq_prepare(H, K, damp, U, dead, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_gptq_quantize_pack(const float* W, int K, int N, const double* U, const unsigned char* dead,
+                          const float* act_sq, const rq_search* search, const rq_packed* out, void* stream) {
+    if (!W || !U || !dead || !out) return RQ_ERR_INVALID_ARG;
+    int s = check_packed(out, K, N);
+    if (s != RQ_OK) return s;
+    if (rq::is_sb(out->fmt)) return RQ_ERR_INVALID_ARG;                  // symmetric formats only
+    if (K > 16384 || rq::gptq_rows_per_block(K, rq::sym_group(out->fmt)) == 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+    rq_search sr = {64, 0.7f, 1.0f};
+    if (search) sr = *search;
+    if (sr.n_cand < 1 || sr.n_cand > 256 || !std::isfinite(sr.t_lo) || !std::isfinite(sr.t_hi) ||
+        !(sr.t_lo > 0.0f) || sr.t_lo > sr.t_hi || sr.t_hi > 4.0f)
+        return RQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(U) || (act_sq && !aligned16(act_sq))) return RQ_ERR_MISALIGNED;
+    size_t sbytes = 0;
+    rq_packed_size(out->fmt, K, N, nullptr, &sbytes);
+    rq::GptqArgs a = {out->fmt, K, N, W, U, dead, act_sq, sr.n_cand, sr.t_lo, sr.t_hi, out->codes, out->scales,
+                      sbytes};
+    return cuda_status(rq::launch_gptq_pack(a, static_cast<cudaStream_t>(stream)));
+}
+
 int rq_wgemm(const void* x, int M, int K, int N, const rq_packed* w, float* y, void* stream) {
     if (!x || !y || !w) return RQ_ERR_INVALID_ARG;
     if (M < 1 || M > 128) return RQ_ERR_INVALID_ARG;
@@ -157,6 +194,7 @@ const char* rq_status_string(int status) {
         case RQ_ERR_MISALIGNED: return "a device pointer is not 16-byte aligned";
         case RQ_ERR_CUDA: return "CUDA runtime error (see rq_last_cuda_error)";
         case RQ_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+        case RQ_ERR_NOT_POSITIVE_DEFINITE: return "a GPTQ Hessian was not positive definite after damping";
         default: return "unknown status";
     }
 }
@@ -166,13 +204,16 @@ int rq_last_cuda_error(void) { return t_last_cuda; }
 int rq_device_status(void* stream, int* word) {
     if (!word) return RQ_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    unsigned a = 0, b = 0, c = 0;
+    unsigned a = 0, b = 0, c = 0, d = 0;
     int s = cuda_status(rq::status_pack(st, &a));
     if (s == RQ_OK) s = cuda_status(rq::status_gemv(st, &b));
     if (s == RQ_OK) s = cuda_status(rq::status_tc(st, &c));
-    *word = (int)(a | b | c);
+    if (s == RQ_OK) s = cuda_status(rq::status_gptq(st, &d));
+    const unsigned w = a | b | c | d;
+    *word = (int)w;
     if (s != RQ_OK) return s;
-    return *word ? RQ_ERR_DEVICE_TIMEOUT : RQ_OK;
+    if (w & ~(unsigned)rq::kStatusNotSpd) return RQ_ERR_DEVICE_TIMEOUT;
+    return w ? RQ_ERR_NOT_POSITIVE_DEFINITE : RQ_OK;
 }
 
 int rq_version(void) { return 100; }

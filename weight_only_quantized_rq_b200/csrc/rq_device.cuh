@@ -24,6 +24,7 @@ enum : unsigned {
     kStatusMmaWait = 1u << 2,    // waited too long for a tensor-core commit
     kStatusTmem = 1u << 3,       // TMEM allocation did not succeed
     kStatusXWait = 1u << 4,      // waited too long for a staged activation buffer
+    // 1u << 5: kStatusNotSpd (rq_internal.h), a Cholesky pivot that was not positive
 };
 
 // One word per translation unit (internal linkage, so no device linking is

@@ -8,6 +8,10 @@
 
 namespace rq {
 
+// Device status bit of a Cholesky pivot that was not positive (the other
+// bits, all bounded-wait timeouts, are listed with the device helpers).
+constexpr unsigned kStatusNotSpd = 1u << 5;
+
 constexpr int kFmtW4G64 = 1;
 constexpr int kFmtW8G16 = 2;
 constexpr int kFmtW4SB32 = 3;
@@ -54,6 +58,25 @@ struct PackArgs {
 };
 
 cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st);
+
+// GPTQ on the preset's grid (symmetric formats): the input Hessian, the
+// upper Cholesky factor U of its damped inverse, and the column loop.
+struct GptqArgs {
+    int fmt, K, N;
+    const float* W;
+    const double* U;
+    const uint8_t* dead;
+    const float* act_sq;
+    int n_cand;
+    float t_lo, t_hi;
+    void* codes;
+    void* scales;
+    size_t scales_bytes;
+};
+cudaError_t launch_hessian(const void* x, int R, int K, double* H, cudaStream_t st);
+cudaError_t launch_gptq_prepare(const double* H, int K, double damp, double* U, uint8_t* dead, cudaStream_t st);
+cudaError_t launch_gptq_pack(const GptqArgs& a, cudaStream_t st);
+int gptq_rows_per_block(int K, int G);   // 0 when one row does not fit in shared memory
 cudaError_t launch_dequant(int fmt, int K, int N, const void* codes, const void* scales, float* out,
                            cudaStream_t st);
 
@@ -86,6 +109,7 @@ cudaError_t launch_act_finalize(const double* sum_sq, int K, long long rows, flo
 
 // Read and clear the device status word of each kernel file (synchronizes st).
 cudaError_t status_pack(cudaStream_t st, unsigned* word);
+cudaError_t status_gptq(cudaStream_t st, unsigned* word);
 cudaError_t status_gemv(cudaStream_t st, unsigned* word);
 cudaError_t status_tc(cudaStream_t st, unsigned* word);
 

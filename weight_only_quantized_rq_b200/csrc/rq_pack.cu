@@ -58,11 +58,49 @@ __device__ __forceinline__ void warp_argmin(double& L, int& idx) {
 }
 
 constexpr int kPackWarps = 8;
+constexpr int kGptqWarps = 8;      // most rows per block of the GPTQ kernel
+
+// Shared memory of one GPTQ row: the row in fp64, its codes, the group's
+// fp32 weights and loss weights.
+__host__ __device__ constexpr size_t gptq_warp_bytes(int K, int G) {
+    return (size_t)K * 8 + (size_t)K + (size_t)G * 8;
+}
 constexpr double kInf = __builtin_huge_val();
 
+// The E[x^2]-weighted search of one symmetric group of G weights held in
+// shared memory by the calling warp (w, and the weights a of the loss):
+// absmax, base = absmax / qmax, candidate i's scale fp16(t_i * base), loss
+// sum_k a_k (w_k - q_k s_i)^2 in fp64 in ascending k, the lowest index with
+// the least loss. Lane l evaluates candidates l, l + 32, ...; every lane
+// returns the chosen scale.
+template <int G>
+__device__ __forceinline__ __half sym_search(const float* w, const float* a, float qmax, int n_cand, float t_lo,
+                                             float t_hi, int lane) {
+    float amax = 0.0f;
+    for (int k = lane; k < G; k += 32) amax = fmaxf(amax, fabsf(w[k]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float base = __fdiv_rn(amax, qmax);
+    if (n_cand == 1) return __float2half_rn(__fmul_rn(cand_t(0, 1, t_lo, t_hi), base));
+    double bestL = kInf;   // lanes without a candidate never win
+    int bestI = 0x7fffffff;
+    for (int i = lane; i < n_cand; i += 32) {
+        const float sf = __half2float(__float2half_rn(__fmul_rn(cand_t(i, n_cand, t_lo, t_hi), base)));
+        double L = 0.0;
+        for (int k = 0; k < G; ++k) {
+            const float wk = w[k];
+            const float wq = __fmul_rn((float)sym_code(wk, sf, qmax), sf);
+            const double d = __dsub_rn((double)wk, (double)wq);
+            L = __dadd_rn(L, __dmul_rn((double)a[k], __dmul_rn(d, d)));
+        }
+        if (bestI == 0x7fffffff || L < bestL) { bestL = L; bestI = i; }
+    }
+    warp_argmin(bestL, bestI);
+    return __float2half_rn(__fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), base));
+}
+
 // One warp per symmetric group of G weights: int4 (G = 64, qmax 7), int8
-// (G = 16 or 64, qmax 127), 6-bit (G = 16, qmax 31). Lane l evaluates
-// candidates l, l+32, ...
+// (G = 16 or 64, qmax 127), 6-bit (G = 16, qmax 31).
 template <int G, int QMAX>
 __global__ void __launch_bounds__(kPackWarps * 32)
 qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
@@ -77,40 +115,13 @@ qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restr
     if (gid >= total) return;
     const int n = (int)(gid / ng), g = (int)(gid % ng);
     const float* w = W + (size_t)n * K + (size_t)g * G;
-
-    float amax = 0.0f;
     for (int k = lane; k < G; k += 32) {
-        const float v = w[k];
-        s_w[warp][k] = v;
+        s_w[warp][k] = w[k];
         s_a[warp][k] = act_sq ? act_sq[(size_t)g * G + k] : 1.0f;
-        amax = fmaxf(amax, fabsf(v));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     __syncwarp();
     const float qmax = (float)QMAX;
-    const float base = __fdiv_rn(amax, qmax);
-
-    __half best_s;
-    if (n_cand == 1) {
-        best_s = __float2half_rn(__fmul_rn(cand_t(0, 1, t_lo, t_hi), base));
-    } else {
-        double bestL = kInf;   // lanes without a candidate never win
-        int bestI = 0x7fffffff;
-        for (int i = lane; i < n_cand; i += 32) {
-            const float sf = __half2float(__float2half_rn(__fmul_rn(cand_t(i, n_cand, t_lo, t_hi), base)));
-            double L = 0.0;
-            for (int k = 0; k < G; ++k) {
-                const float wk = s_w[warp][k];
-                const float wq = __fmul_rn((float)sym_code(wk, sf, qmax), sf);
-                const double d = __dsub_rn((double)wk, (double)wq);
-                L = __dadd_rn(L, __dmul_rn((double)s_a[warp][k], __dmul_rn(d, d)));
-            }
-            if (bestI == 0x7fffffff || L < bestL) { bestL = L; bestI = i; }
-        }
-        warp_argmin(bestL, bestI);
-        best_s = __float2half_rn(__fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), base));
-    }
+    const __half best_s = sym_search<G>(s_w[warp], s_a[warp], qmax, n_cand, t_lo, t_hi, lane);
     const float sf = __half2float(best_s);
     if (QMAX == 7) {
         // lane l writes byte l of the group: k = 2l (low nibble), 2l+1 (high)
@@ -142,6 +153,78 @@ qpack_sym_kernel(const float* __restrict__ W, int K, int N, const float* __restr
         }
     }
     if (lane == 0) scales[(size_t)n * ng + g] = __half_as_ushort(best_s);
+}
+
+// GPTQ on the preset's grid for a symmetric format (GPTQ, Frantar et al.
+// 2022; rwkv-quant article, "Calibration leakage and honest measurements"):
+// one warp per row, the row held in fp64 in shared memory. Columns in order;
+// at each group's first column the group's scale is the preset's search on
+// fp32 of the current weights; then per column k:
+//   q_k = clamp(rint(fp32(w_k) / s), -qmax, qmax),
+//   err = (w_k - q_k s) / U[k][k],  w_j = w_j - err * U[k][j] for j > k
+// (fp64, one rounding per operation, lanes over j; the updates of each w_j
+// arrive in ascending k). Dead columns start at 0. The codes are emitted at
+// the end in the format's layout.
+template <int G, int QMAX>
+__global__ void __launch_bounds__(kGptqWarps * 32)
+gptq_sym_kernel(const float* __restrict__ W, int K, int N, const double* __restrict__ U,
+                const uint8_t* __restrict__ dead, const float* __restrict__ act_sq, int n_cand, float t_lo,
+                float t_hi, uint8_t* __restrict__ codes, uint16_t* __restrict__ scales) {
+    extern __shared__ __align__(16) uint8_t g_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * (int)(blockDim.x >> 5) + warp;
+    if (n >= N) return;
+    const size_t per = gptq_warp_bytes(K, G);
+    double* w = reinterpret_cast<double*>(g_smem + (size_t)warp * per);
+    int8_t* q = reinterpret_cast<int8_t*>(w + K);
+    float* wg = reinterpret_cast<float*>(q + K);          // K % 64 == 0: 4-byte aligned
+    float* ag = wg + G;
+    for (int k = lane; k < K; k += 32) w[k] = dead[k] ? 0.0 : (double)W[(size_t)n * K + k];
+    __syncwarp();
+    const float qmax = (float)QMAX;
+    const int ng = K / G;
+    for (int g = 0; g < ng; ++g) {
+        const int k0 = g * G;
+        for (int i = lane; i < G; i += 32) {
+            wg[i] = __double2float_rn(w[k0 + i]);
+            ag[i] = act_sq ? act_sq[k0 + i] : 1.0f;
+        }
+        __syncwarp();
+        const __half sh = sym_search<G>(wg, ag, qmax, n_cand, t_lo, t_hi, lane);
+        if (lane == 0) scales[(size_t)n * ng + g] = __half_as_ushort(sh);
+        const float sf = __half2float(sh);
+        for (int i = 0; i < G; ++i) {
+            const int k = k0 + i;
+            const double wk = w[k];
+            const int qk = sym_code(__double2float_rn(wk), sf, qmax);
+            if (lane == 0) q[k] = (int8_t)qk;
+            const double err = __ddiv_rn(__dsub_rn(wk, (double)__fmul_rn((float)qk, sf)), U[(size_t)k * K + k]);
+            const double* Uk = U + (size_t)k * K;
+            for (int j = k + 1 + lane; j < K; j += 32) w[j] = __dsub_rn(w[j], __dmul_rn(err, Uk[j]));
+            __syncwarp();
+        }
+    }
+    __syncwarp();
+    if (QMAX == 7) {
+        for (int t = lane; t < K / 2; t += 32)
+            codes[(size_t)n * (K / 2) + t] = (uint8_t)((q[2 * t] + 8) | ((q[2 * t + 1] + 8) << 4));
+    } else if (QMAX == 127) {
+        for (int k = lane; k < K; k += 32) codes[(size_t)n * K + k] = (uint8_t)(q[k] + 128);
+    } else {
+        // 6 bits: per 64-weight chunk, bytes 0..31 low nibbles, 32..47 bits 4..5
+        uint8_t* row = codes + (size_t)n * (K / 64 * 48);
+        for (int b = lane; b < K / 64 * 48; b += 32) {
+            const int c = b / 48, o = b - c * 48, j0 = 64 * c;
+            uint32_t v = 0;
+            if (o < 32) {
+                v = (uint32_t)((q[j0 + 2 * o] + 32) & 15) | ((uint32_t)((q[j0 + 2 * o + 1] + 32) & 15) << 4);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v |= (uint32_t)((q[j0 + 4 * (o - 32) + e] + 32) >> 4) << (2 * e);
+            }
+            row[b] = (uint8_t)v;
+        }
+    }
 }
 
 // One block per superblock of 256 weights with BITS-bit codes (4, 5, 6):
@@ -410,6 +493,38 @@ cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st) {
         zero_bytes_kernel<<<1, 32, 0, st>>>(static_cast<uint8_t*>(a.scales) + used, (int)(a.scales_bytes - used));
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+    }
+    pack_done_kernel<<<1, 32, 0, st>>>();
+    return cudaGetLastError();
+}
+
+// Rows per block: as many as fit in 200 KB of shared memory (at most 8).
+int gptq_rows_per_block(int K, int G) {
+    const size_t per = gptq_warp_bytes(K, G);
+    int w = kGptqWarps;
+    while (w > 1 && (size_t)w * per > 200 * 1024) --w;
+    return (size_t)w * per <= 200 * 1024 ? w : 0;
+}
+
+cudaError_t launch_gptq_pack(const GptqArgs& a, cudaStream_t st) {
+    const int G = sym_group(a.fmt);
+    const int rows = gptq_rows_per_block(a.K, G);
+    if (rows == 0) return cudaErrorInvalidValue;
+    auto kern = a.fmt == kFmtW4G64 ? gptq_sym_kernel<64, 7>
+              : a.fmt == kFmtW8G16 ? gptq_sym_kernel<16, 127>
+              : a.fmt == kFmtW8G64 ? gptq_sym_kernel<64, 127>
+                                   : gptq_sym_kernel<16, 31>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    const size_t smem = (size_t)rows * gptq_warp_bytes(a.K, G);
+    kern<<<(unsigned)((a.N + rows - 1) / rows), rows * 32, smem, st>>>(
+        a.W, a.K, a.N, a.U, a.dead, a.act_sq, a.n_cand, a.t_lo, a.t_hi, static_cast<uint8_t*>(a.codes),
+        static_cast<uint16_t*>(a.scales));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t used = (size_t)a.N * (a.K / G) * 2;
+    if (a.scales_bytes > used) {
+        zero_bytes_kernel<<<1, 32, 0, st>>>(static_cast<uint8_t*>(a.scales) + used, (int)(a.scales_bytes - used));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     pack_done_kernel<<<1, 32, 0, st>>>();
     return cudaGetLastError();

@@ -452,6 +452,46 @@ def run_ours(args, w, M):
                                   "note": "algorithmic bytes = R * K * 2 (x read once) per call"},
                      "kernel": "act_sumsq_kernel"}
         del xa, ss
+    # GPTQ on the preset grid for one 1.5B projection (2048 -> 2048, int4 g64)
+    # from 4096 calibration rows: the three device steps, each timed alone
+    gptq = None
+    if not args.quick:
+        K_g, N_g, R_g = 2048, 2048, 4096
+        g_g = torch.Generator(device=dev).manual_seed(91)
+        basis = torch.randn(256, K_g, device=dev, generator=g_g)
+        xg = (torch.randn(R_g, 256, device=dev, generator=g_g) @ basis
+              + 0.1 * torch.randn(R_g, K_g, device=dev, generator=g_g)).to(torch.bfloat16)
+        Wg = torch.randn(N_g, K_g, device=dev, generator=g_g) * 0.02
+        Hg = torch.zeros(K_g, K_g, dtype=torch.float64, device=dev)
+        Ug = torch.empty(K_g, K_g, dtype=torch.float64, device=dev)
+        dg = torch.empty(K_g, dtype=torch.uint8, device=dev)
+        outg = rq.alloc_packed("w4g64", K_g, N_g, dev)
+
+        def ev_time(fn, reps):
+            with torch.cuda.stream(stream):
+                fn()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    fn()
+                e1.record(stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        ms_h = ev_time(lambda: rq.rq_hessian_accum(xg, Hg, stream=stream), 3)
+        Hg.zero_()
+        rq.rq_hessian_accum(xg, Hg, stream=stream)
+        ms_p = ev_time(lambda: rq.rq_gptq_prepare(Hg, 0.01, Ug, dg, stream=stream), 2)
+        ms_q = ev_time(lambda: rq.rq_gptq_quantize_pack(Wg, "w4g64", Ug, dg, None, 64, 0.7, 1.0, outg,
+                                                        stream=stream), 2)
+        gptq = {"K": K_g, "N": N_g, "rows": R_g, "fmt": "w4g64",
+                "hessian_ms": round(ms_h, 3), "hessian_fp64_TFLOP_s": round(2.0 * K_g * K_g * R_g / (ms_h * 1e-3) / 1e12, 2),
+                "prepare_ms": round(ms_p, 3), "pack_ms": round(ms_q, 3),
+                "pack_fp64_GFLOP_s": round(N_g * K_g * K_g / (ms_q * 1e-3) / 1e9, 1),
+                "kernels": "hessian_kernel; gptq_reverse/chol_col (one launch per column)/chol_diag/trinv/"
+                           "gptq_finish; gptq_sym_kernel",
+                "note": "offline calibration steps, measured for reference; not part of the decode step"}
+        del xg, Wg, Hg, Ug, dg, outg, basis
     status = rq.rq_device_status(stream)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
@@ -477,6 +517,7 @@ def run_ours(args, w, M):
                         "flops / bf16 peak) divided by the step time",
         "preset_variants": variants,
         "act_stats": act_stats,
+        "gptq": gptq,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": prob.h2d,
                 "d2h_bytes_per_step": prob.d2h},

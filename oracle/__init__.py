@@ -88,6 +88,8 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_hessian_accum.restype = None
     L.orc_gptq_pack_sym.argtypes = [_P, _i, _i, _P, _P, _P, _i, _i, _f, _f, _P, _P]
     L.orc_gptq_pack_sym.restype = None
+    L.orc_gptq_pack_sb.argtypes = [_P, _i, _i, _P, _P, _P, _i, _f, _f, _i, _P]
+    L.orc_gptq_pack_sb.restype = None
     L.orc_threads.argtypes = []
     L.orc_threads.restype = _i
     L.orc_set_threads.argtypes = [_i]
@@ -314,17 +316,19 @@ def gptq_prepare(H, damp: float = 0.01):
 
 
 def gptq_pack(fmt: str, W, U, dead, act_sq=None, n_cand: int = 64, t_lo: float = 0.7, t_hi: float = 1.0):
-    """GPTQ on the preset's grid for a symmetric format; the same planes as
-    pack(). Returns (codes, scales)."""
+    """GPTQ on the preset's grid; the same planes as pack(). Returns
+    (codes, scales or None)."""
     W = _c(W, np.float32)
     N, K = W.shape
     U = _c(U, np.float64)
     dead = _c(dead, np.uint8)
     a = None if act_sq is None else _c(act_sq, np.float32)
     cshape, cdt, sshape = packed_shapes(fmt, K, N)
-    if sshape is None:
-        raise ValueError("GPTQ is built for the symmetric formats")
     codes = np.zeros(cshape, dtype=cdt)
+    if fmt in SB_BITS:
+        lib().orc_gptq_pack_sb(_ptr(W), K, N, _ptr(U), _ptr(dead), _ptr(a), n_cand, t_lo, t_hi, SB_BITS[fmt],
+                               _ptr(codes))
+        return codes, None
     scales = np.zeros(sshape, dtype=np.uint16)
     lib().orc_gptq_pack_sym(_ptr(W), K, N, _ptr(U), _ptr(dead), _ptr(a), FORMATS[fmt], n_cand, t_lo, t_hi,
                             _ptr(codes), _ptr(scales))

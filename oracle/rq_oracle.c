@@ -448,6 +448,17 @@ int orc_asym_group(const float *w, const float *a, int G, const float *t, int n,
  * The final codes use the stored values S_j = d * sc_j and M_j = dmin * m_j
  * (both exact fp32 products); there is no second search after the 6-bit
  * rounding. */
+/* Put code q of weight kk (0..255) into a record whose code area starts
+ * zeroed: the low 4 bits in the nibble bytes, bits 4.. in the plane. */
+static void sb_put_code(uint8_t *blk, int kk, int q, int bits)
+{
+    int lo4 = q & 15, up = q >> 4;
+    if ((kk & 1) == 0) blk[16 + kk / 2] = (uint8_t)lo4;
+    else blk[16 + kk / 2] |= (uint8_t)(lo4 << 4);
+    if (bits == 5) blk[144 + kk / 8] |= (uint8_t)(up << (kk % 8));
+    if (bits == 6) blk[144 + kk / 4] |= (uint8_t)(up << (2 * (kk % 4)));
+}
+
 void orc_sb_finish(const float *w, const float *S_star, const float *M_star, int bits, uint8_t *blk)
 {
     const int levels = (1 << bits) - 1;
@@ -479,18 +490,62 @@ void orc_sb_finish(const float *w, const float *S_star, const float *M_star, int
         float M = dm * (float)mc[j];
         for (int k = 0; k < 32; k++) {
             int kk = 32 * j + k;
-            int q = asym_code(w[kk], S, M, levels);
-            int lo4 = q & 15, up = q >> 4;
-            if ((kk & 1) == 0) blk[16 + kk / 2] = (uint8_t)lo4;
-            else blk[16 + kk / 2] |= (uint8_t)(lo4 << 4);
-            if (bits == 5) blk[144 + kk / 8] |= (uint8_t)(up << (kk % 8));
-            if (bits == 6) blk[144 + kk / 4] |= (uint8_t)(up << (2 * (kk % 4)));
+            sb_put_code(blk, kk, asym_code(w[kk], S, M, levels), bits);
         }
     }
 }
 
 /* Pack a whole [N][K] matrix (K % 256 == 0) into [N][K/256] superblocks of
  * `bits`-bit codes. */
+int orc_sb_field(const uint8_t *blk, int which, int j);
+
+/* GPTQ into the asymmetric superblock formats (the COMPRESSION preset's
+ * grid): at each superblock's first column the eight groups' (S*, M*) come
+ * from the preset's search (orc_asym_group) on fp32 of the current weights and
+ * the record's header is formed as orc_sb_finish forms it; the stored
+ * S_j = d sc_j, M_j = dmin m_j are then fixed and the superblock's 256 columns
+ * are quantized in order with GPTQ's error feedback:
+ *   q = asym_code(fp32(w_k), S_j, M_j),  w_hat = fp32(S_j q) - M_j,
+ *   err = (w_k - w_hat) / U[k][k],  w_j -= err * U[k][j] for j > k (fp64).
+ * U and dead as for orc_gptq_pack_sym. */
+void orc_gptq_pack_sb(const float *W, int K, int N, const double *U, const uint8_t *dead, const float *a,
+                      int n_cand, float t_lo, float t_hi, int bits, uint8_t *blocks)
+{
+    int nb = K / 256;
+    int levels = (1 << bits) - 1;
+    size_t rs = (size_t)sb_bytes(bits);
+    float *t = (float *)malloc(sizeof(float) * (size_t)n_cand);
+    orc_grid(n_cand, t_lo, t_hi, t);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < N; n++) {
+        double *w = (double *)malloc(sizeof(double) * (size_t)K);
+        for (int k = 0; k < K; k++) w[k] = dead[k] ? 0.0 : (double)W[(size_t)n * K + k];
+        for (int b = 0; b < nb; b++) {
+            int k0 = b * 256;
+            float wsb[256], S[8], M[8];
+            for (int i = 0; i < 256; i++) wsb[i] = (float)w[k0 + i];
+            for (int j = 0; j < 8; j++)
+                orc_asym_group(wsb + 32 * j, a ? a + k0 + 32 * j : NULL, 32, t, n_cand, bits, &S[j], &M[j], NULL);
+            uint8_t *blk = blocks + ((size_t)n * nb + b) * rs;
+            orc_sb_finish(wsb, S, M, bits, blk);
+            memset(blk + 16, 0, rs - 16);
+            float d = orc_f16_to_f32((uint16_t)(blk[0] | (blk[1] << 8)));
+            float dm = orc_f16_to_f32((uint16_t)(blk[2] | (blk[3] << 8)));
+            for (int i = 0; i < 256; i++) {
+                int k = k0 + i;
+                float Sj = d * (float)orc_sb_field(blk, 0, i / 32);
+                float Mj = dm * (float)orc_sb_field(blk, 1, i / 32);
+                int q = asym_code((float)w[k], Sj, Mj, levels);
+                sb_put_code(blk, i, q, bits);
+                double err = (w[k] - (double)asym_deq(q, Sj, Mj)) / U[(size_t)k * K + k];
+                for (int j = k + 1; j < K; j++) w[j] = w[j] - err * U[(size_t)k * K + j];
+            }
+        }
+        free(w);
+    }
+    free(t);
+}
+
 void orc_pack_sb32(const float *W, int K, int N, const float *a, int n_cand,
                    float t_lo, float t_hi, int bits, uint8_t *blocks)
 {

@@ -50,6 +50,10 @@ MUTANTS = [
      "for (int i = 0; i < G; i++) wg[i] = W[(size_t)n * K + k0 + i];", None),
     ("GPTQ keeps dead columns", "w[k] = dead[k] ? 0.0 : (double)W[(size_t)n * K + k];", "w[k] = (double)W[(size_t)n * K + k];", None),
     ("GPTQ code from the group search's codes", "int q = sym_code((float)w[k], sf, qmax);", "int q = qg[i];", None),
+    ("GPTQ superblock header from the original weights", "for (int i = 0; i < 256; i++) wsb[i] = (float)w[k0 + i];",
+     "for (int i = 0; i < 256; i++) wsb[i] = W[(size_t)n * K + k0 + i];", None),
+    ("GPTQ superblock error without the min", "double err = (w[k] - (double)asym_deq(q, Sj, Mj)) / U[(size_t)k * K + k];",
+     "double err = (w[k] - (double)((float)q * Sj)) / U[(size_t)k * K + k];", None),
     ("Hessian skips the last row", "for (int r = 0; r < R; r++) {\n                double xi", "for (int r = 0; r < R - 1; r++) {\n                double xi", None),
     ("E[x^2] sums |x| instead of x^2", "part = part + v * v;", "part = part + fabs(v);", None),
     ("E[x^2] skips the last chunk", "for (int c = 0; c < 64; c++) {\n            int r0", "for (int c = 0; c < 63; c++) {\n            int r0", None),

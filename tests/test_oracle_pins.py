@@ -685,3 +685,80 @@ def test_gptq_lowers_the_output_error(orc):
         D = W.astype(np.float64) - orc.dequant("w4g64", K, N, c, s).astype(np.float64)
         return float(np.einsum("nk,kl,nl->", D, H, D))
     assert out_err(cg, sg) < 0.7 * out_err(cr, sr)
+
+
+def _gptq_sb_by_obs(orc, fmt, W, H, a, n_cand, damp=0.01):
+    """Superblock GPTQ written the second way (explicit inverse of the
+    trailing Hessian block): returns w_hat [N][K] and the records' headers."""
+    bits = orc.SB_BITS[fmt]
+    L = (1 << bits) - 1
+    N, K = W.shape
+    Hd = np.array(H, dtype=np.float64, copy=True)
+    dead = np.diag(Hd) == 0
+    Hd[dead, dead] = 1.0
+    Hd[np.arange(K), np.arange(K)] += damp * np.mean(np.diag(Hd))
+    what = np.zeros((N, K), np.float64)
+    headers = np.zeros((N, K // 256, 16), np.uint8)
+    for n in range(N):
+        w = W[n].astype(np.float64)
+        w[dead] = 0.0
+        for b in range(K // 256):
+            k0 = 256 * b
+            wsb = w[k0:k0 + 256].astype(np.float32)
+            S = np.zeros(8, np.float32)
+            M = np.zeros(8, np.float32)
+            for j in range(8):
+                _, S[j], M[j], _ = orc.asym_group(wsb[32 * j:32 * j + 32],
+                                                  None if a is None else a[k0 + 32 * j:k0 + 32 * j + 32],
+                                                  n_cand, bits=bits)
+            blk = orc.sb_finish(wsb, S, M, bits)
+            headers[n, b] = blk[:16]
+            d, dm = orc.f16_bits_to_f32(blk[:4].copy().view(np.uint16))
+            for i in range(256):
+                k = k0 + i
+                Sj = np.float32(d * np.float32(orc.sb_field(blk, 0, i // 32)))
+                Mj = np.float32(dm * np.float32(orc.sb_field(blk, 1, i // 32)))
+                if Sj == 0:
+                    q = 0
+                else:
+                    v = np.float32(np.float32(np.float32(w[k]) + Mj) / Sj)
+                    q = int(np.rint(np.clip(v, np.float32(0), np.float32(L))))
+                wq = float(np.float32(np.float32(np.float32(q) * Sj) - Mj))
+                what[n, k] = wq
+                e = w[k] - wq
+                Hinv = np.linalg.inv(Hd[k:, k:])
+                w[k:] -= e * Hinv[:, 0] / Hinv[0, 0]
+    return what, headers
+
+
+@pytest.mark.parametrize("fmt", ["w4sb32", "w5sb32", "w6sb32"])
+def test_gptq_sb_matches_sequential_obs(orc, fmt):
+    rng = np.random.default_rng(79)
+    N, K, R = 2, 512, 900
+    mix = rng.standard_normal((K, K)) * 0.2 + np.eye(K)
+    x = (rng.standard_normal((R, K)) @ mix).astype(np.float32)
+    H = orc.hessian_accum(_bf16_bits(x))
+    a = (np.diag(H) / R).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    U, dead = orc.gptq_prepare(H)
+    codes, _ = orc.gptq_pack(fmt, W, U, dead, a, n_cand=16)
+    what, headers = _gptq_sb_by_obs(orc, fmt, W, H, a, 16)
+    rs = orc.SB_BYTES[fmt]
+    assert np.array_equal(codes.reshape(N, K // 256, rs)[:, :, :16], headers)
+    assert np.array_equal(orc.dequant(fmt, K, N, codes, None).astype(np.float64), what)
+
+
+@pytest.mark.parametrize("fmt", ["w4sb32", "w6sb32"])
+def test_gptq_sb_diagonal_hessian_is_the_preset_pack(orc, fmt):
+    rng = np.random.default_rng(83)
+    N, K = 3, 512
+    d = rng.random(K) * 3 + 0.5
+    d[300] = 0.0
+    U, dead = orc.gptq_prepare(np.diag(d))
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    a = rng.random(K).astype(np.float32) + 0.1
+    c1, _ = orc.gptq_pack(fmt, W, U, dead, a, n_cand=32)
+    W0 = W.copy()
+    W0[:, 300] = 0.0
+    c0, _ = orc.pack(fmt, W0, a, n_cand=32)
+    assert np.array_equal(c1, c0)

@@ -266,13 +266,19 @@ int rq_hessian_accum(const void *x, int R, int K, double *H, void *stream);
  * rq_device_status) and leaves NaNs in U. Limits: 1 <= K <= 16384. */
 int rq_gptq_prepare(const double *H, int K, double damp, double *U, unsigned char *dead, void *stream);
 
-/* rq_gptq_quantize_pack: quantize W into `out` (a symmetric format:
- * RQ_W4_SYM_G64, RQ_W8_SYM_G16, RQ_W8_SYM_G64 or RQ_W6_SYM_G16; the same
- * planes as rq_quantize_pack). Per row, in fp64, columns in order: dead
- * columns start at 0; at each group's first column the group's scale is
- * rq_quantize_pack's search (act_sq, search as there) on the group's current
- * weights rounded to fp32; then q_k = clamp(rint(fp32(w_k) / s), +-qmax),
- * err = (w_k - q_k s) / U[k][k] and w_j -= err * U[k][j] for j > k.
+/* rq_gptq_quantize_pack: quantize W into `out` (any format; the same
+ * planes as rq_quantize_pack). Per row, in fp64, columns in order; dead
+ * columns start at 0.
+ *   Symmetric formats: at each group's first column the group's scale is
+ *   rq_quantize_pack's search (act_sq, search as there) on the group's
+ *   current weights rounded to fp32; then q_k = clamp(rint(fp32(w_k) / s),
+ *   +-qmax) and w_hat_k = q_k s.
+ *   Superblock formats: at each superblock's first column its eight groups
+ *   are searched and its header (d, dmin, 6-bit fields) formed as
+ *   rq_quantize_pack does, on the current weights rounded to fp32; then
+ *   q_k = clamp(rint((fp32(w_k) + M_j) / S_j), 0, 2^b - 1) with the stored
+ *   S_j, M_j and w_hat_k = fp32(S_j q_k) - M_j.
+ * In both: err = (w_k - w_hat_k) / U[k][k] and w_j -= err * U[k][j] for j > k.
  *   W device fp32 [N][K]; U, dead from rq_gptq_prepare. K <= 16384.
  * Same ordering rules as rq_quantize_pack. */
 int rq_gptq_quantize_pack(const float *W, int K, int N, const double *U, const unsigned char *dead,

@@ -137,8 +137,9 @@ def test_gptq_validation(L):
     assert L.rq_gptq_prepare(U, 64, 0.01, B, B, st) == rq.RQ_ERR_MISALIGNED
     d = _desc("w4g64", 2048, 64)
     assert L.rq_gptq_quantize_pack(A, 2048, 64, None, B, None, None, ctypes.byref(d), st) == rq.RQ_ERR_INVALID_ARG
-    sb = _desc("w4sb32", 2048, 64, scales=0)
-    assert L.rq_gptq_quantize_pack(A, 2048, 64, B, B, None, None, ctypes.byref(sb), st) == rq.RQ_ERR_INVALID_ARG
+    sb = _desc("w4sb32", 2048, 64)                          # superblock descriptor with a scales plane
+    assert L.rq_gptq_quantize_pack(A, 2048, 64, B, B, None, None, ctypes.byref(sb), st) == rq.RQ_ERR_FORMAT_MISMATCH
+    assert L.rq_gptq_quantize_pack(A, 2048, 64, B, B, U, None, ctypes.byref(d), st) == rq.RQ_ERR_MISALIGNED
     wide = _desc("w4g64", 32768, 4)
     assert L.rq_gptq_quantize_pack(A, 32768, 4, B, B, None, None, ctypes.byref(wide), st) == rq.RQ_ERR_UNSUPPORTED_SHAPE
     assert L.rq_gptq_quantize_pack(A, 1024, 64, B, B, None, None, ctypes.byref(d), st) == rq.RQ_ERR_FORMAT_MISMATCH

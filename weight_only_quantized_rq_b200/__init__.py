@@ -305,9 +305,9 @@ def rq_gptq_prepare(H: torch.Tensor, damp: float = 0.01, U: torch.Tensor | None 
 def rq_gptq_quantize_pack(W: torch.Tensor, fmt, U: torch.Tensor, dead: torch.Tensor,
                           act_sq: torch.Tensor | None = None, n_cand: int = 64, t_lo: float = 0.7, t_hi: float = 1.0,
                           out: Packed | None = None, stream=None) -> Packed:
-    """GPTQ on the preset's grid: quantize W (fp32 [N][K], CUDA) into a
-    symmetric format with the factor of rq_gptq_prepare. Returns the Packed
-    matrix (same planes as rq_quantize_pack)."""
+    """GPTQ on the preset's grid: quantize W (fp32 [N][K], CUDA) into any
+    format with the factor of rq_gptq_prepare. Returns the Packed matrix (same
+    planes as rq_quantize_pack)."""
     N, K = W.shape
     if out is None:
         out = alloc_packed(fmt, K, N, W.device)

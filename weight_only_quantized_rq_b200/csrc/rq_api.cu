@@ -117,8 +117,7 @@ int rq_gptq_quantize_pack(const float* W, int K, int N, const double* U, const u
     if (!W || !U || !dead || !out) return RQ_ERR_INVALID_ARG;
     int s = check_packed(out, K, N);
     if (s != RQ_OK) return s;
-    if (rq::is_sb(out->fmt)) return RQ_ERR_INVALID_ARG;                  // symmetric formats only
-    if (K > 16384 || rq::gptq_rows_per_block(K, rq::sym_group(out->fmt)) == 0) return RQ_ERR_UNSUPPORTED_SHAPE;
+    if (K > 16384 || rq::gptq_rows_per_block(out->fmt, K) == 0) return RQ_ERR_UNSUPPORTED_SHAPE;
     rq_search sr = {64, 0.7f, 1.0f};
     if (search) sr = *search;
     if (sr.n_cand < 1 || sr.n_cand > 256 || !std::isfinite(sr.t_lo) || !std::isfinite(sr.t_hi) ||

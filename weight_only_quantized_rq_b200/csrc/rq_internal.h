@@ -59,8 +59,8 @@ struct PackArgs {
 
 cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st);
 
-// GPTQ on the preset's grid (symmetric formats): the input Hessian, the
-// upper Cholesky factor U of its damped inverse, and the column loop.
+// GPTQ on the preset's grid (every format): the input Hessian, the upper
+// Cholesky factor U of its damped inverse, and the column loop.
 struct GptqArgs {
     int fmt, K, N;
     const float* W;
@@ -76,7 +76,7 @@ struct GptqArgs {
 cudaError_t launch_hessian(const void* x, int R, int K, double* H, cudaStream_t st);
 cudaError_t launch_gptq_prepare(const double* H, int K, double damp, double* U, uint8_t* dead, cudaStream_t st);
 cudaError_t launch_gptq_pack(const GptqArgs& a, cudaStream_t st);
-int gptq_rows_per_block(int K, int G);   // 0 when one row does not fit in shared memory
+int gptq_rows_per_block(int fmt, int K);   // 0 when one row does not fit in shared memory
 cudaError_t launch_dequant(int fmt, int K, int N, const void* codes, const void* scales, float* out,
                            cudaStream_t st);
 

@@ -65,6 +65,11 @@ constexpr int kGptqWarps = 8;      // most rows per block of the GPTQ kernel
 __host__ __device__ constexpr size_t gptq_warp_bytes(int K, int G) {
     return (size_t)K * 8 + (size_t)K + (size_t)G * 8;
 }
+// Superblock formats: the record (208 bytes at most), 32 scale/min floats,
+// the superblock's 256 weights and loss weights, the row in fp64.
+__host__ __device__ constexpr size_t gptq_sb_warp_bytes(int K) {
+    return 208 + 32 * 4 + 512 * 4 + (size_t)K * 8;
+}
 constexpr double kInf = __builtin_huge_val();
 
 // The E[x^2]-weighted search of one symmetric group of G weights held in
@@ -227,9 +232,101 @@ gptq_sym_kernel(const float* __restrict__ W, int K, int N, const double* __restr
     }
 }
 
+// The preset's search for one asymmetric group of 32 weights held in shared
+// memory by the calling warp (w, and the loss weights a): lo = min(0, min w),
+// hi = max(0, max w); candidate i shrinks [lo, hi] about its midpoint by t_i
+// (r = t_i (hi - lo) / 2, S = 2 r / (2^b - 1), M = max(0, r - mid)); loss as
+// for the symmetric search; lowest index with the least loss. Every lane
+// returns the chosen (S*, M*).
+template <int BITS>
+__device__ __forceinline__ void asym_search(const float* w, const float* a, int n_cand, float t_lo, float t_hi,
+                                            int lane, float& S_out, float& M_out) {
+    constexpr float kTop = (float)((1 << BITS) - 1);        // highest code
+    float lo = w[lane] < 0.0f ? w[lane] : 0.0f;
+    float hi = w[lane] > 0.0f ? w[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+        const float h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+        lo = l2 < lo ? l2 : lo;
+        hi = h2 > hi ? h2 : hi;
+    }
+    const float half = __fmul_rn(__fsub_rn(hi, lo), 0.5f);
+    const float mid = __fmul_rn(__fadd_rn(hi, lo), 0.5f);
+    double bestL = kInf;
+    int bestI = 0x7fffffff;
+    for (int i = lane; i < n_cand; i += 32) {
+        const float r = __fmul_rn(cand_t(i, n_cand, t_lo, t_hi), half);
+        const float S = __fdiv_rn(__fmul_rn(2.0f, r), kTop);
+        const float loi = __fsub_rn(mid, r);
+        const float M = loi < 0.0f ? -loi : 0.0f;
+        double loss = 0.0;
+        if (n_cand > 1) {
+            for (int k = 0; k < 32; ++k) {
+                const float wk = w[k];
+                const float wq = __fsub_rn(__fmul_rn((float)asym_code(wk, S, M, kTop), S), M);
+                const double d = __dsub_rn((double)wk, (double)wq);
+                loss = __dadd_rn(loss, __dmul_rn((double)a[k], __dmul_rn(d, d)));
+            }
+        }
+        if (bestI == 0x7fffffff || loss < bestL) { bestL = loss; bestI = i; }
+    }
+    warp_argmin(bestL, bestI);
+    const float r = __fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), half);
+    const float loi = __fsub_rn(mid, r);
+    S_out = __fdiv_rn(__fmul_rn(2.0f, r), kTop);
+    M_out = loi < 0.0f ? -loi : 0.0f;
+}
+
+// A record's header from the eight groups' (S*, M*) (shared memory s_S,
+// s_M), by one warp: d = fp16(max S* / 63), dmin = fp16(max M* / 63), 6-bit
+// sc_j = rint(S*_j / d), m_j = rint(M*_j / dmin) (0 when d or dmin is 0),
+// the stored S_j = d sc_j, M_j = dmin m_j into s_Sq, s_Mq, and the 16 header
+// bytes (fp16 d, fp16 dmin, the 96-bit field string) into s_blk.
+__device__ __forceinline__ void sb_header(const float* s_S, const float* s_M, int lane, float* s_Sq, float* s_Mq,
+                                          uint8_t* s_blk) {
+    float mS = 0.0f, mM = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        mS = s_S[j] > mS ? s_S[j] : mS;
+        mM = s_M[j] > mM ? s_M[j] : mM;
+    }
+    const __half dh = __float2half_rn(__fdiv_rn(mS, 63.0f));
+    const __half mh = __float2half_rn(__fdiv_rn(mM, 63.0f));
+    const float d = __half2float(dh), dm = __half2float(mh);
+    uint32_t field = 0;   // lanes 0..7: sc_j, lanes 8..15: m_j
+    if (lane < 16) {
+        const int j = lane & 7;
+        const float num = lane < 8 ? s_S[j] : s_M[j];
+        const float den = lane < 8 ? d : dm;
+        field = den == 0.0f ? 0u : (uint32_t)(int)rintf(clampf(__fdiv_rn(num, den), 0.0f, 63.0f));
+        if (lane < 8) s_Sq[j] = __fmul_rn(d, (float)field);
+        else s_Mq[j] = __fmul_rn(dm, (float)field);
+    }
+    // assemble the 96-bit string: field f (0..15) at bit 6f
+    uint32_t words[3] = {0u, 0u, 0u};
+#pragma unroll
+    for (int f = 0; f < 16; ++f) {
+        const uint64_t v = (uint64_t)__shfl_sync(0xffffffffu, field, f);
+        const int bit = 6 * f;
+        const int wi = bit >> 5, sh = bit & 31;
+        const uint64_t placed = v << sh;
+        words[wi] |= (uint32_t)placed;
+        if (wi + 1 < 3) words[wi + 1] |= (uint32_t)(placed >> 32);
+    }
+    if (lane == 0) {
+        uint32_t* hdr = reinterpret_cast<uint32_t*>(s_blk);
+        hdr[0] = (uint32_t)__half_as_ushort(dh) | ((uint32_t)__half_as_ushort(mh) << 16);
+        hdr[1] = words[0];
+        hdr[2] = words[1];
+        hdr[3] = words[2];
+    }
+}
+
 // One block per superblock of 256 weights with BITS-bit codes (4, 5, 6):
-// warp j searches group j (32 weights), then the block forms d, dmin, the
-// 6-bit fields, the codes' low nibbles and (5, 6 bits) the high-bit plane.
+// warp j searches group j (32 weights), then warp 0 forms d, dmin, the 6-bit
+// fields, and the block the codes' low nibbles and (5, 6 bits) the high-bit
+// plane.
 template <int BITS>
 __global__ void __launch_bounds__(256)
 qpack_sb_kernel(const float* __restrict__ W, int K, int N, const float* __restrict__ act_sq,
@@ -250,87 +347,16 @@ qpack_sb_kernel(const float* __restrict__ W, int K, int N, const float* __restri
     s_w[t] = W[(size_t)n * K + k0 + t];
     s_a[t] = act_sq ? act_sq[k0 + t] : 1.0f;
     __syncthreads();
-
     {   // group search (warp = group j)
-        const float* w = s_w + 32 * warp;
-        const float* a = s_a + 32 * warp;
-        float lo = w[lane] < 0.0f ? w[lane] : 0.0f;
-        float hi = w[lane] > 0.0f ? w[lane] : 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float l2 = __shfl_xor_sync(0xffffffffu, lo, o);
-            const float h2 = __shfl_xor_sync(0xffffffffu, hi, o);
-            lo = l2 < lo ? l2 : lo;
-            hi = h2 > hi ? h2 : hi;
-        }
-        const float half = __fmul_rn(__fsub_rn(hi, lo), 0.5f);
-        const float mid = __fmul_rn(__fadd_rn(hi, lo), 0.5f);
-        double bestL = kInf;
-        int bestI = 0x7fffffff;
-        for (int i = lane; i < n_cand; i += 32) {
-            const float r = __fmul_rn(cand_t(i, n_cand, t_lo, t_hi), half);
-            const float S = __fdiv_rn(__fmul_rn(2.0f, r), kTop);
-            const float loi = __fsub_rn(mid, r);
-            const float M = loi < 0.0f ? -loi : 0.0f;
-            double loss = 0.0;
-            if (n_cand > 1) {
-                for (int k = 0; k < 32; ++k) {
-                    const float wk = w[k];
-                    const float wq = __fsub_rn(__fmul_rn((float)asym_code(wk, S, M, kTop), S), M);
-                    const double d = __dsub_rn((double)wk, (double)wq);
-                    loss = __dadd_rn(loss, __dmul_rn((double)a[k], __dmul_rn(d, d)));
-                }
-            }
-            if (bestI == 0x7fffffff || loss < bestL) { bestL = loss; bestI = i; }
-        }
-        warp_argmin(bestL, bestI);
+        float S, M;
+        asym_search<BITS>(s_w + 32 * warp, s_a + 32 * warp, n_cand, t_lo, t_hi, lane, S, M);
         if (lane == 0) {
-            const float r = __fmul_rn(cand_t(bestI, n_cand, t_lo, t_hi), half);
-            const float loi = __fsub_rn(mid, r);
-            s_S[warp] = __fdiv_rn(__fmul_rn(2.0f, r), kTop);
-            s_M[warp] = loi < 0.0f ? -loi : 0.0f;
+            s_S[warp] = S;
+            s_M[warp] = M;
         }
     }
     __syncthreads();
-
-    if (warp == 0) {   // superblock scale/min and the 6-bit fields
-        float mS = 0.0f, mM = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            mS = s_S[j] > mS ? s_S[j] : mS;
-            mM = s_M[j] > mM ? s_M[j] : mM;
-        }
-        const __half dh = __float2half_rn(__fdiv_rn(mS, 63.0f));
-        const __half mh = __float2half_rn(__fdiv_rn(mM, 63.0f));
-        const float d = __half2float(dh), dm = __half2float(mh);
-        uint32_t field = 0;   // lanes 0..7: sc_j, lanes 8..15: m_j
-        if (lane < 16) {
-            const int j = lane & 7;
-            const float num = lane < 8 ? s_S[j] : s_M[j];
-            const float den = lane < 8 ? d : dm;
-            field = den == 0.0f ? 0u : (uint32_t)(int)rintf(clampf(__fdiv_rn(num, den), 0.0f, 63.0f));
-            if (lane < 8) s_Sq[j] = __fmul_rn(d, (float)field);
-            else s_Mq[j] = __fmul_rn(dm, (float)field);
-        }
-        // assemble the 96-bit string: field f (0..15) at bit 6f
-        uint32_t words[3] = {0u, 0u, 0u};
-#pragma unroll
-        for (int f = 0; f < 16; ++f) {
-            const uint64_t v = (uint64_t)__shfl_sync(0xffffffffu, field, f);
-            const int bit = 6 * f;
-            const int wi = bit >> 5, sh = bit & 31;
-            const uint64_t placed = v << sh;
-            words[wi] |= (uint32_t)placed;
-            if (wi + 1 < 3) words[wi + 1] |= (uint32_t)(placed >> 32);
-        }
-        if (lane == 0) {
-            uint32_t* hdr = reinterpret_cast<uint32_t*>(s_blk);
-            hdr[0] = (uint32_t)__half_as_ushort(dh) | ((uint32_t)__half_as_ushort(mh) << 16);
-            hdr[1] = words[0];
-            hdr[2] = words[1];
-            hdr[3] = words[2];
-        }
-    }
+    if (warp == 0) sb_header(s_S, s_M, lane, s_Sq, s_Mq, s_blk);
     __syncthreads();
     s_q[t] = (uint8_t)asym_code(s_w[t], s_Sq[t >> 5], s_Mq[t >> 5], kTop);   // code of weight t
     __syncthreads();
@@ -353,6 +379,76 @@ qpack_sb_kernel(const float* __restrict__ W, int K, int N, const float* __restri
     if (t < RS / 16) {
         uint4* dst = reinterpret_cast<uint4*>(blocks + ((size_t)n * nb + b) * RS);
         dst[t] = reinterpret_cast<const uint4*>(s_blk)[t];
+    }
+}
+
+// GPTQ into the asymmetric superblock formats: one warp per row, the row in
+// fp64 in shared memory. At each superblock's first column: the eight group
+// searches on fp32 of the current weights and the record's header (the same
+// helpers as qpack_sb_kernel); then the superblock's 256 columns in order:
+//   q = asym_code(fp32(w_k), S_j, M_j), w_hat = fp32(S_j q) - M_j,
+//   err = (w_k - w_hat) / U[k][k],  w_j = w_j - err * U[k][j] for j > k.
+template <int BITS>
+__global__ void __launch_bounds__(kGptqWarps * 32)
+gptq_sb_kernel(const float* __restrict__ W, int K, int N, const double* __restrict__ U,
+               const uint8_t* __restrict__ dead, const float* __restrict__ act_sq, int n_cand, float t_lo,
+               float t_hi, uint8_t* __restrict__ blocks) {
+    constexpr int RS = 16 + 128 + (BITS - 4) * 32;
+    constexpr float kTop = (float)((1 << BITS) - 1);
+    extern __shared__ __align__(16) uint8_t g_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * (int)(blockDim.x >> 5) + warp;
+    if (n >= N) return;
+    uint8_t* base = g_smem + (size_t)warp * gptq_sb_warp_bytes(K);
+    uint8_t* blk = base;                                           // RS bytes (16-byte aligned)
+    float* S = reinterpret_cast<float*>(base + 208);               // S*[8], M*[8], Sq[8], Mq[8]
+    float* M = S + 8;
+    float* Sq = S + 16;
+    float* Mq = S + 24;
+    float* wsb = S + 32;                                           // 256 fp32 weights
+    float* asb = wsb + 256;                                        // 256 loss weights
+    double* w = reinterpret_cast<double*>(asb + 256);              // the row
+    for (int k = lane; k < K; k += 32) w[k] = dead[k] ? 0.0 : (double)W[(size_t)n * K + k];
+    __syncwarp();
+    const int nb = K / 256;
+    for (int b = 0; b < nb; ++b) {
+        const int k0 = 256 * b;
+        for (int i = lane; i < 256; i += 32) {
+            wsb[i] = __double2float_rn(w[k0 + i]);
+            asb[i] = act_sq ? act_sq[k0 + i] : 1.0f;
+        }
+        __syncwarp();
+        for (int j = 0; j < 8; ++j) {
+            float Sj, Mj;
+            asym_search<BITS>(wsb + 32 * j, asb + 32 * j, n_cand, t_lo, t_hi, lane, Sj, Mj);
+            if (lane == 0) {
+                S[j] = Sj;
+                M[j] = Mj;
+            }
+        }
+        __syncwarp();
+        sb_header(S, M, lane, Sq, Mq, blk);
+        for (int i = 16 + lane; i < RS; i += 32) blk[i] = 0;
+        __syncwarp();
+        for (int i = 0; i < 256; ++i) {
+            const int k = k0 + i, j = i >> 5;
+            const double wk = w[k];
+            const int q = asym_code(__double2float_rn(wk), Sq[j], Mq[j], kTop);
+            if (lane == 0) {                                       // low nibble, then the plane bits
+                if ((i & 1) == 0) blk[16 + i / 2] = (uint8_t)(q & 15);
+                else blk[16 + i / 2] |= (uint8_t)((q & 15) << 4);
+                if (BITS == 5) blk[144 + i / 8] |= (uint8_t)((q >> 4) << (i % 8));
+                if (BITS == 6) blk[144 + i / 4] |= (uint8_t)((q >> 4) << (2 * (i % 4)));
+            }
+            const float wq = __fsub_rn(__fmul_rn((float)q, Sq[j]), Mq[j]);
+            const double err = __ddiv_rn(__dsub_rn(wk, (double)wq), U[(size_t)k * K + k]);
+            const double* Uk = U + (size_t)k * K;
+            for (int j2 = k + 1 + lane; j2 < K; j2 += 32) w[j2] = __dsub_rn(w[j2], __dmul_rn(err, Uk[j2]));
+            __syncwarp();
+        }
+        uint4* dst = reinterpret_cast<uint4*>(blocks + ((size_t)n * nb + b) * RS);
+        if (lane < RS / 16) dst[lane] = reinterpret_cast<const uint4*>(blk)[lane];
+        __syncwarp();
     }
 }
 
@@ -499,17 +595,28 @@ cudaError_t launch_quantize_pack(const PackArgs& a, cudaStream_t st) {
 }
 
 // Rows per block: as many as fit in 200 KB of shared memory (at most 8).
-int gptq_rows_per_block(int K, int G) {
-    const size_t per = gptq_warp_bytes(K, G);
+int gptq_rows_per_block(int fmt, int K) {
+    const size_t per = is_sb(fmt) ? gptq_sb_warp_bytes(K) : gptq_warp_bytes(K, sym_group(fmt));
     int w = kGptqWarps;
     while (w > 1 && (size_t)w * per > 200 * 1024) --w;
     return (size_t)w * per <= 200 * 1024 ? w : 0;
 }
 
 cudaError_t launch_gptq_pack(const GptqArgs& a, cudaStream_t st) {
-    const int G = sym_group(a.fmt);
-    const int rows = gptq_rows_per_block(a.K, G);
+    const int rows = gptq_rows_per_block(a.fmt, a.K);
     if (rows == 0) return cudaErrorInvalidValue;
+    if (is_sb(a.fmt)) {
+        auto kern = a.fmt == kFmtW4SB32 ? gptq_sb_kernel<4> : a.fmt == kFmtW5SB32 ? gptq_sb_kernel<5>
+                                                                               : gptq_sb_kernel<6>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)((a.N + rows - 1) / rows), rows * 32, (size_t)rows * gptq_sb_warp_bytes(a.K), st>>>(
+            a.W, a.K, a.N, a.U, a.dead, a.act_sq, a.n_cand, a.t_lo, a.t_hi, static_cast<uint8_t*>(a.codes));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        pack_done_kernel<<<1, 32, 0, st>>>();
+        return cudaGetLastError();
+    }
+    const int G = sym_group(a.fmt);
     auto kern = a.fmt == kFmtW4G64 ? gptq_sym_kernel<64, 7>
               : a.fmt == kFmtW8G16 ? gptq_sym_kernel<16, 127>
               : a.fmt == kFmtW8G64 ? gptq_sym_kernel<64, 127>

@@ -192,7 +192,8 @@ int rq_wgemm(const void *x, int M, int K, int N, const rq_packed *w, float *y, v
 typedef struct rq_wgemm_item {
     const void *x;          /* device bf16 [M][K] */
     const rq_packed *w;     /* packed matrix (host descriptor) */
-    float *y;               /* device fp32 [M][N], overwritten */
+    void *y;                /* device [M][N], overwritten: fp32 (rq_wgemm_batch,
+                               RQ_OUT_F32) or bf16 (RQ_OUT_BF16) */
 } rq_wgemm_item;
 
 /* `count` independent products in ONE launch, e.g. the r, k and v
@@ -209,6 +210,22 @@ typedef struct rq_wgemm_item {
  * and ordering rules as rq_wgemm (the packed planes must not be written by
  * the kernel launched just before this call on the stream). */
 int rq_wgemm_batch(const rq_wgemm_item *items, int count, int M, void *stream);
+
+/* Output element types of rq_wgemm_out / rq_wgemm_batch_out. */
+typedef enum rq_out_type {
+    RQ_OUT_F32 = 0,         /* fp32, as rq_wgemm */
+    RQ_OUT_BF16 = 1         /* the fp32 result rounded once to bf16 (nearest even) */
+} rq_out_type;
+
+/* rq_wgemm / rq_wgemm_batch with the output element type chosen: y is fp32
+ * [M][N] (RQ_OUT_F32) or bf16 [M][N] (RQ_OUT_BF16). The bf16 result is
+ * exactly the RQ_OUT_F32 result rounded to nearest even, written by the same
+ * launch (no second pass over y): the bf16-output epilogue of the batched
+ * r/k/v launch ([rwkv_quant_nv] "Operator Optimization Details"). Same
+ * validation and ordering rules as rq_wgemm; any other out_type is
+ * RQ_ERR_INVALID_ARG. */
+int rq_wgemm_out(const void *x, int M, int K, int N, const rq_packed *w, void *y, int out_type, void *stream);
+int rq_wgemm_batch_out(const rq_wgemm_item *items, int count, int M, int out_type, void *stream);
 
 /* Export w_hat as fp32 [N][K] into W_out (device).  ([CARD] summary: the
  * kernel output is bit-identical to the offline dequantization.) Uses the

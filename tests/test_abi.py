@@ -147,6 +147,17 @@ def test_gptq_validation(L):
     assert rq.rq_status_string(rq.RQ_ERR_NOT_POSITIVE_DEFINITE) != "unknown status"
 
 
+def test_wgemm_out_validation(L):
+    d = _desc("w4g64", 2048, 256)
+    st = ctypes.c_void_p(0)
+    assert L.rq_wgemm_out(A, 1, 2048, 256, ctypes.byref(d), A, 2, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_wgemm_out(A, 1, 2048, 256, ctypes.byref(d), A, -1, st) == rq.RQ_ERR_INVALID_ARG
+    assert L.rq_wgemm_out(A, 1, 2048, 256, ctypes.byref(d), U, rq.RQ_OUT_BF16, st) == rq.RQ_ERR_MISALIGNED
+    item = rq.RqWgemmItem(0x40000, ctypes.pointer(d), 0x40000)
+    arr = (rq.RqWgemmItem * 1)(item)
+    assert L.rq_wgemm_batch_out(arr, 1, 1, 3, st) == rq.RQ_ERR_INVALID_ARG
+
+
 def test_dequant_validation(L):
     st = ctypes.c_void_p(0)
     d = _desc("w4sb32", 512, 8, scales=0)

@@ -366,3 +366,49 @@ def test_wgemm_batch_equals_single_calls():
     torch.cuda.synchronize()
     for a, b in zip(ys, singles):
         assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------ bf16 output ---
+@pytest.mark.parametrize("fmt,K,N,M", [
+    ("w4g64", 2048, 300, 1),       # register path
+    ("w8g16", 2048, 129, 2),
+    ("w4sb32", 2560, 77, 1),
+    ("w8g64", 1024, 64, 2),
+    ("w4g64", 2048, 300, 16),      # tensor-core epilogue
+    ("w8g16", 448, 33, 128),
+    ("w4sb32", 2560, 300, 8),
+    ("w5sb32", 2560, 99, 1),
+    ("w6g16", 768, 200, 5),
+    ("w4g64", 4096, 200, 24),      # K split over a cluster (rank-order DSMEM reduction)
+    ("w4g64", 4096, 203, 40),      # the same with N % 4 != 0 (element stores)
+])
+def test_wgemm_bf16_output_is_the_rounded_fp32(fmt, K, N, M):
+    """The bf16-output epilogue writes exactly the fp32 result rounded to
+    nearest even, and nothing outside y."""
+    W = wl.random_matrix(3100 + K + N, N, K).cuda()
+    p = rq.rq_quantize_pack(W, fmt, None, 8)
+    x, _ = make_x(3200 + M, M, K)
+    xd = x.cuda()
+    y32 = rq.rq_wgemm(xd, p)
+    big = torch.full((M * N + 512,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y16 = big[256:256 + M * N].view(M, N)
+    rq.rq_wgemm(xd, p, y16)
+    torch.cuda.synchronize()
+    assert torch.equal(y16.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16))
+    assert bool(torch.isnan(big[:256]).all()) and bool(torch.isnan(big[256 + M * N:]).all())
+
+
+@pytest.mark.parametrize("fmt,M", [("w4g64", 1), ("w4g64", 16), ("w8g16", 4)])
+def test_wgemm_batch_bf16_output(fmt, M):
+    """r/k/v-style batch (three 2048^2 products) with bf16 outputs."""
+    xs, ws, y32s, y16s = [], [], [], []
+    for i in range(3):
+        ws.append(rq.rq_quantize_pack(wl.random_matrix(3300 + i, 2048, 2048).cuda(), fmt, None, 4))
+        xs.append(make_x(3400 + i, M, 2048)[0].cuda())
+        y32s.append(torch.empty(M, 2048, device="cuda"))
+        y16s.append(torch.empty(M, 2048, dtype=torch.bfloat16, device="cuda"))
+    rq.rq_wgemm_batch(xs, ws, y32s)
+    rq.rq_wgemm_batch(xs, ws, y16s)
+    torch.cuda.synchronize()
+    for a, b in zip(y16s, y32s):
+        assert torch.equal(a.view(torch.int16), b.to(torch.bfloat16).view(torch.int16))

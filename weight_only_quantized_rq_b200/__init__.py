@@ -33,6 +33,9 @@ RQ_ERR_CUDA = 5
 RQ_ERR_DEVICE_TIMEOUT = 6
 RQ_ERR_NOT_POSITIVE_DEFINITE = 7
 
+RQ_OUT_F32 = 0
+RQ_OUT_BF16 = 1
+
 RQ_W4_SYM_G64 = 1
 RQ_W8_SYM_G16 = 2
 RQ_W4_ASYM_SB32 = 3
@@ -44,7 +47,8 @@ FORMAT_IDS = {"w4g64": RQ_W4_SYM_G64, "w8g16": RQ_W8_SYM_G16, "w4sb32": RQ_W4_AS
               "w5sb32": RQ_W5_ASYM_SB32, "w6sb32": RQ_W6_ASYM_SB32, "w8g64": RQ_W8_SYM_G64,
               "w6g16": RQ_W6_SYM_G16}
 SB_FORMATS = (RQ_W4_ASYM_SB32, RQ_W5_ASYM_SB32, RQ_W6_ASYM_SB32)
-EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_dequant",
+EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_wgemm_out", "rq_wgemm_batch_out",
+           "rq_dequant",
            "rq_act_sumsq", "rq_act_finalize", "rq_hessian_accum", "rq_gptq_prepare", "rq_gptq_quantize_pack",
            "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
 MAX_BATCH = 160
@@ -105,6 +109,10 @@ def _lib() -> ctypes.CDLL:
         L.rq_wgemm.restype = I
         L.rq_wgemm_batch.argtypes = [ctypes.POINTER(RqWgemmItem), I, I, P]
         L.rq_wgemm_batch.restype = I
+        L.rq_wgemm_out.argtypes = [P, I, I, I, ctypes.POINTER(RqPacked), P, I, P]
+        L.rq_wgemm_out.restype = I
+        L.rq_wgemm_batch_out.argtypes = [ctypes.POINTER(RqWgemmItem), I, I, I, P]
+        L.rq_wgemm_batch_out.restype = I
         L.rq_dequant.argtypes = [ctypes.POINTER(RqPacked), P, P]
         L.rq_dequant.restype = I
         L.rq_act_sumsq.argtypes = [P, I, I, P, P]
@@ -210,14 +218,24 @@ def rq_quantize_pack(W: torch.Tensor, fmt, act_sq: torch.Tensor | None = None, n
     return out
 
 
-def rq_wgemm(x: torch.Tensor, w: Packed, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y = x @ w_hat.T with x bf16 [M][K] and y fp32 [M][N] (CUDA tensors)."""
+def _out_type(dtype) -> int:
+    if dtype == torch.float32:
+        return RQ_OUT_F32
+    if dtype == torch.bfloat16:
+        return RQ_OUT_BF16
+    raise ValueError("y must be float32 or bfloat16")
+
+
+def rq_wgemm(x: torch.Tensor, w: Packed, y: torch.Tensor | None = None, stream=None,
+             out_dtype=torch.float32) -> torch.Tensor:
+    """y = x @ w_hat.T with x bf16 [M][K] and y [M][N] (CUDA tensors), y fp32
+    or bf16 (the fp32 result rounded once; by y's dtype, else out_dtype)."""
     M, K = x.shape
     if y is None:
-        y = torch.empty(M, w.N, dtype=torch.float32, device=x.device)
+        y = torch.empty(M, w.N, dtype=out_dtype, device=x.device)
     d = w.desc()
-    _check(_lib().rq_wgemm(_ptr(x), int(M), int(K), int(w.N), ctypes.byref(d), _ptr(y), _stream(stream)),
-           "rq_wgemm")
+    _check(_lib().rq_wgemm_out(_ptr(x), int(M), int(K), int(w.N), ctypes.byref(d), _ptr(y), _out_type(y.dtype),
+                               _stream(stream)), "rq_wgemm_out")
     return y
 
 
@@ -232,14 +250,18 @@ class WgemmBatch:
         self._keep = (list(xs), list(ws), list(ys))
         self._descs = [w.desc() for w in ws]
         self._items = (RqWgemmItem * len(xs))()
+        self.out = _out_type(ys[0].dtype)
         for i, (x, d, y) in enumerate(zip(xs, self._descs, ys)):
             if int(x.shape[0]) != self.M:
                 raise ValueError("every item must have the same M")
+            if _out_type(y.dtype) != self.out:
+                raise ValueError("every y must have the same dtype")
             self._items[i] = RqWgemmItem(x.data_ptr(), ctypes.pointer(d), y.data_ptr())
         self.count = len(xs)
 
     def __call__(self, stream=None):
-        _check(_lib().rq_wgemm_batch(self._items, self.count, self.M, _stream(stream)), "rq_wgemm_batch")
+        _check(_lib().rq_wgemm_batch_out(self._items, self.count, self.M, self.out, _stream(stream)),
+               "rq_wgemm_batch_out")
 
 
 def rq_wgemm_batch(xs, ws, ys, stream=None) -> None:

@@ -131,21 +131,27 @@ int rq_gptq_quantize_pack(const float* W, int K, int N, const double* U, const u
     return cuda_status(rq::launch_gptq_pack(a, static_cast<cudaStream_t>(stream)));
 }
 
-int rq_wgemm(const void* x, int M, int K, int N, const rq_packed* w, float* y, void* stream) {
+int rq_wgemm_out(const void* x, int M, int K, int N, const rq_packed* w, void* y, int out_type, void* stream) {
     if (!x || !y || !w) return RQ_ERR_INVALID_ARG;
     if (M < 1 || M > 128) return RQ_ERR_INVALID_ARG;
+    if (out_type != RQ_OUT_F32 && out_type != RQ_OUT_BF16) return RQ_ERR_INVALID_ARG;
     int s = check_packed(w, K, N);
     if (s != RQ_OK) return s;
     if (!aligned16(x) || !aligned16(y)) return RQ_ERR_MISALIGNED;
-    rq::WgemmArgs a = {w->fmt, M, K, N, x, w->codes, w->scales, y};
+    rq::WgemmArgs a = {w->fmt, M, K, N, x, w->codes, w->scales, y, out_type == RQ_OUT_BF16 ? 1 : 0};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (rq::tc_supported(w->fmt, M)) return cuda_status(rq::launch_tc(&a, 1, st));
     return cuda_status(rq::launch_gemv(&a, 1, st));
 }
 
-int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
+int rq_wgemm(const void* x, int M, int K, int N, const rq_packed* w, float* y, void* stream) {
+    return rq_wgemm_out(x, M, K, N, w, y, RQ_OUT_F32, stream);
+}
+
+int rq_wgemm_batch_out(const rq_wgemm_item* items, int count, int M, int out_type, void* stream) {
     if (!items || count < 1 || count > rq::kMaxBatch) return RQ_ERR_INVALID_ARG;
     if (M < 1 || M > 128) return RQ_ERR_INVALID_ARG;
+    if (out_type != RQ_OUT_F32 && out_type != RQ_OUT_BF16) return RQ_ERR_INVALID_ARG;
     rq::WgemmArgs a[rq::kMaxBatch];
     for (int i = 0; i < count; ++i) {
         const rq_wgemm_item& it = items[i];
@@ -154,11 +160,15 @@ int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
         if (s != RQ_OK) return s;
         if (it.w->fmt != items[0].w->fmt) return RQ_ERR_FORMAT_MISMATCH;
         if (!aligned16(it.x) || !aligned16(it.y)) return RQ_ERR_MISALIGNED;
-        a[i] = {it.w->fmt, M, it.w->K, it.w->N, it.x, it.w->codes, it.w->scales, it.y};
+        a[i] = {it.w->fmt, M, it.w->K, it.w->N, it.x, it.w->codes, it.w->scales, it.y, out_type == RQ_OUT_BF16 ? 1 : 0};
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (rq::tc_supported(a[0].fmt, M)) return cuda_status(rq::launch_tc(a, count, st));
     return cuda_status(rq::launch_gemv(a, count, st));
+}
+
+int rq_wgemm_batch(const rq_wgemm_item* items, int count, int M, void* stream) {
+    return rq_wgemm_batch_out(items, count, M, RQ_OUT_F32, stream);
 }
 
 int rq_dequant(const rq_packed* w, float* W_out, void* stream) {

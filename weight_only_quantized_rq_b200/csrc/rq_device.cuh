@@ -27,6 +27,12 @@ enum : unsigned {
     // 1u << 5: kStatusNotSpd (rq_internal.h), a Cholesky pivot that was not positive
 };
 
+// Output element idx of y: fp32, or rounded once to bf16 (nearest even).
+__device__ __forceinline__ void store_y(void* y, size_t idx, float v, int bf16) {
+    if (bf16) static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
+    else static_cast<float*>(y)[idx] = v;
+}
+
 // One word per translation unit (internal linkage, so no device linking is
 // needed); each kernel file exports a host accessor that reads and clears it.
 static __device__ unsigned g_status = 0u;

@@ -64,7 +64,8 @@ struct Item {                  // one product of a launch
     const uint16_t* x;         // bf16 bits [M][K]
     const uint8_t* codes;
     const uint8_t* scales;
-    float* y;                  // fp32 [M][N]
+    void* y;                   // fp32 [M][N], or bf16 when ybf16
+    int ybf16;
     long long cost0;           // packed bytes of the items before this one
     long long cost1;           // cost0 + this item's packed bytes
     int K, N;
@@ -460,7 +461,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             const int rr = rbase + r;
             if ((lane & 7) == 0 && rr < rg) {
                 if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = v;
-                else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = v;
+                else if (m < mrows) store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, v, it.ybf16);
             }
         }
     } else {                                             // shuffle tree per row, lane 0 of each team stores
@@ -480,7 +481,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = yacc[r][m];
-                        else if (m < mrows) it.y[(size_t)(m0 + m) * it.N + g0 + rr] = yacc[r][m];
+                        else if (m < mrows) store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, yacc[r][m], it.ybf16);
                     }
             }
         }
@@ -533,7 +534,7 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
                         const float* q = red + ((size_t)rr * MT + m) * KS;
                         float v = 0.0f;
                         for (int k = 0; k < KS; ++k) v += q[k];
-                        it.y[(size_t)(m0 + m) * it.N + g0 + rr] = v;
+                        store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, v, it.ybf16);
                     }
                 }
             }
@@ -832,6 +833,7 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
             it.codes = static_cast<const uint8_t*>(a[i].codes);
             it.scales = static_cast<const uint8_t*>(a[i].scales);
             it.y = a[i].y;
+            it.ybf16 = a[i].ybf16;
             it.cost0 = total;
             const long long U = (it.N + it.rho - 1) / it.rho;
             total += U * it.ucost;

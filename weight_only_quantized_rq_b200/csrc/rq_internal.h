@@ -85,7 +85,8 @@ struct WgemmArgs {
     const void* x;         // bf16 [M][K]
     const void* codes;
     const void* scales;
-    float* y;              // fp32 [M][N]
+    void* y;               // fp32 [M][N], or bf16 [M][N] when ybf16
+    int ybf16;             // 1: y is rounded once to bf16 (round to nearest even)
 };
 
 // Memory-bound path (few activation rows): dequantize in registers, fp32

@@ -95,7 +95,8 @@ struct __align__(64) TcItem {       // one product of a launch
     CUtensorMap cmap;               // codes plane: uint8 [N][crb], box [128 rows][RB bytes], swizzled
     CUtensorMap xmap;               // x: bf16 [M][K] viewed as [K/64][M][64], box [KS/64][xrows][64]
     const uint8_t* scales;          // fp16 [N][K / G]
-    float* y;                       // fp32 [M][N]
+    void* y;                        // fp32 [M][N], or bf16 when ybf16
+    int ybf16;
     int K, N, T;                    // T = stages = ceil(K / KS)
     int unit0;                      // index of this product's first tile
     uint32_t srb;                   // scale bytes per row
@@ -816,7 +817,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             tc_fence_after();
             const TcItem& it = p.it[u.item];
             const int N = it.N, n = u.n0 + r;
-            float* y = it.y;
+            void* y = it.y;
             const uint32_t dc = tmem + tl + (uint32_t)(d * niss * Mpad);
             for (int c0 = 0; c0 < Mpad; c0 += 16) {
                 float v[16];
@@ -834,7 +835,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 } else if (n < N) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c0 + j < M) y[(size_t)(c0 + j) * N + n] = v[j];
+                        if (c0 + j < M) store_y(y, (size_t)(c0 + j) * N + n, v[j], it.ybf16);
                 }
             }
             tc_fence_before();
@@ -861,14 +862,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
             }
             const int n = n0 + r4;
-            float* yr = it.y + (size_t)m * N;
+            const size_t row = (size_t)m * N;
             if ((N & 3) == 0 && n + 3 < N) {
-                *reinterpret_cast<float4*>(yr + n) = s;
+                if (it.ybf16) {
+                    const __nv_bfloat162 lo = __floats2bfloat162_rn(s.x, s.y), hi = __floats2bfloat162_rn(s.z, s.w);
+                    uint2 u;
+                    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+                    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+                    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(it.y) + row + n) = u;
+                } else {
+                    *reinterpret_cast<float4*>(static_cast<float*>(it.y) + row + n) = s;
+                }
             } else {
-                if (n < N) yr[n] = s.x;
-                if (n + 1 < N) yr[n + 1] = s.y;
-                if (n + 2 < N) yr[n + 2] = s.z;
-                if (n + 3 < N) yr[n + 3] = s.w;
+                if (n < N) store_y(it.y, row + n, s.x, it.ybf16);
+                if (n + 1 < N) store_y(it.y, row + n + 1, s.y, it.ybf16);
+                if (n + 2 < N) store_y(it.y, row + n + 2, s.z, it.ybf16);
+                if (n + 3 < N) store_y(it.y, row + n + 3, s.w, it.ybf16);
             }
         }
         cluster_sync();                                     // peers have finished reading this CTA
@@ -952,6 +961,7 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
             return cudaErrorInvalidValue;
         it.scales = static_cast<const uint8_t*>(w.scales);
         it.y = w.y;
+        it.ybf16 = w.ybf16;
         it.K = w.K;
         it.N = w.N;
         it.T = (w.K + KS - 1) / KS;

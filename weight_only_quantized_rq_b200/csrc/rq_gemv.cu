@@ -64,8 +64,7 @@ struct Item {                  // one product of a launch
     const uint16_t* x;         // bf16 bits [M][K]
     const uint8_t* codes;
     const uint8_t* scales;
-    void* y;                   // fp32 [M][N], or bf16 when ybf16
-    int ybf16;
+    void* y;                   // fp32 [M][N], or bf16 (the kernel's YB)
     long long cost0;           // packed bytes of the items before this one
     long long cost1;           // cost0 + this item's packed bytes
     int K, N;
@@ -256,7 +255,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& c, int i) {
 // Rows past rg (the group's last rows) lie inside the stage buffer, which
 // always has room for Rg rows; they hold stale bytes whose results are never
 // stored.
-template <int FMT, int MT, int RW, int TT>
+template <int FMT, int MT, int RW, int TT, int YB>
 __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0, int rg, uint32_t x_s, int m0, int mrows, int lane, int rbase, int slice,
                                            float* red) {
     constexpr bool kW4 = !is_w8(FMT);
@@ -461,7 +460,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
             const int rr = rbase + r;
             if ((lane & 7) == 0 && rr < rg) {
                 if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = v;
-                else if (m < mrows) store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, v, it.ybf16);
+                else if (m < mrows) store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, v, YB);
             }
         }
     } else {                                             // shuffle tree per row, lane 0 of each team stores
@@ -481,7 +480,7 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         if (it.KS > 1) red[((size_t)rr * MT + m) * it.KS + slice] = yacc[r][m];
-                        else if (m < mrows) store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, yacc[r][m], it.ybf16);
+                        else if (m < mrows) store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, yacc[r][m], YB);
                     }
             }
         }
@@ -505,7 +504,7 @@ struct Ring {
 // team's slice-0 warp adds the k-slices after a team barrier) and releases
 // the stage. The launch shape (RW, TT) is fixed per item, so the per-item
 // setup stays outside the group loop. False if a bounded wait gave up.
-template <int FMT, int MT, int RW, int TT>
+template <int FMT, int MT, int RW, int TT, int YB>
 __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& ring, uint32_t x_s, int m0,
                                           int mrows, int warp, int lane) {
     const int T = TT ? TT : it.T, KS = it.KS, Rg = it.Rg;
@@ -524,7 +523,7 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
         const int rg = min(Rg, rb - g0);
         if (wfirst < rg) {                               // warp-uniform
             float* red = reinterpret_cast<float*>(ring.red + (size_t)s * ring.red_bytes);
-            gemv_group<FMT, MT, RW, TT>(it, ring.base + (uint32_t)s * ring.stage_bytes, g0, rg, x_s, m0, mrows,
+            gemv_group<FMT, MT, RW, TT, YB>(it, ring.base + (uint32_t)s * ring.stage_bytes, g0, rg, x_s, m0, mrows,
                                         lane, rbase, slice, red);
             if (KS > 1) {
                 asm volatile("bar.sync %0, %1;" :: "r"(1 + team), "r"(KS * 32) : "memory");
@@ -534,7 +533,7 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
                         const float* q = red + ((size_t)rr * MT + m) * KS;
                         float v = 0.0f;
                         for (int k = 0; k < KS; ++k) v += q[k];
-                        store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, v, it.ybf16);
+                        store_y(it.y, (size_t)(m0 + m) * it.N + g0 + rr, v, YB);
                     }
                 }
             }
@@ -548,7 +547,8 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
 // Resident CTAs per SM the register budget is sized for.
 constexpr int min_blocks(int) { return kConsumerWarps <= 12 ? 2 : 1; }
 
-template <int FMT, int MT, int MAXI>
+// YB: outputs rounded once to bf16 (1) or fp32 (0), fixed per launch.
+template <int FMT, int MT, int MAXI, int YB>
 __global__ void __launch_bounds__(kThreads, min_blocks(MT))
 gemv_kernel(const Batch<MAXI> p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -670,13 +670,13 @@ gemv_kernel(const Batch<MAXI> p) {
         const uint32_t x_s = smem_s + p.x_off + (uint32_t)b * p.x_bytes;
         bool ok;
         if (it.T == 32) {                                // whole-warp teams: the common case
-            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 32>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 32>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                              : gemv_item<FMT, MT, 1, 32>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
+            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                              : gemv_item<FMT, MT, 1, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
         } else {
-            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 0>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 0>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                              : gemv_item<FMT, MT, 1, 0>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
+            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
+                              : gemv_item<FMT, MT, 1, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
         }
         if (!ok) return;
         __syncwarp();
@@ -702,9 +702,9 @@ constexpr size_t kSmemBatch = RQ_GEMV_SMEM_BATCH_KB * 1024;
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemAttr = kSmemLimit + 1024;
 
-template <int FMT, int MT, int MAXI>
+template <int FMT, int MT, int MAXI, int YB>
 cudaError_t launch_one(const Batch<MAXI>& prm, size_t smem, int grid, cudaStream_t st) {
-    auto kern = gemv_kernel<FMT, MT, MAXI>;
+    auto kern = gemv_kernel<FMT, MT, MAXI, YB>;
     // The attribute is per device; set it once per device (a race between
     // host threads only repeats the same idempotent call).
     static unsigned long long attr_done = 0ull;
@@ -833,7 +833,6 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
             it.codes = static_cast<const uint8_t*>(a[i].codes);
             it.scales = static_cast<const uint8_t*>(a[i].scales);
             it.y = a[i].y;
-            it.ybf16 = a[i].ybf16;
             it.cost0 = total;
             const long long U = (it.N + it.rho - 1) / it.rho;
             total += U * it.ucost;
@@ -874,8 +873,11 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
         for (int m0 = 0; m0 < M; m0 += MT) {
             p.m0 = m0;
             p.mrows = M - m0 < MT ? M - m0 : MT;
-            const cudaError_t e = MT == 2 ? launch_one<FMT, 2, MAXI>(p, smem, grid, st)
-                                          : launch_one<FMT, 1, MAXI>(p, smem, grid, st);
+            const bool yb = a[0].ybf16 != 0;
+            const cudaError_t e = MT == 2 ? (yb ? launch_one<FMT, 2, MAXI, 1>(p, smem, grid, st)
+                                                : launch_one<FMT, 2, MAXI, 0>(p, smem, grid, st))
+                                          : (yb ? launch_one<FMT, 1, MAXI, 1>(p, smem, grid, st)
+                                                : launch_one<FMT, 1, MAXI, 0>(p, smem, grid, st));
             if (e != cudaSuccess) return e;
         }
         return cudaSuccess;

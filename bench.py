@@ -62,6 +62,23 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(ms: float, ws: int, device) -> float:
+    """The largest of the ranks' times (every rank takes part, in the same
+    order, whatever its value)."""
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(ws: int, bytes_per_rank: float, ms_max: float) -> float:
+    """Weak scaling: every rank streams bytes_per_rank per step; the job's
+    rate is all ranks' bytes over the slowest rank's step time."""
+    return ws * bytes_per_rank / (ms_max * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------- clocks -------
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region."""
@@ -361,21 +378,16 @@ def run_ours(args, w, M):
                 fn()
             e1.record(stream)
         barrier()
-        ms = e0.elapsed_time(e1) / steps
-        t = torch.tensor([ms], device=dev)
-        if ws > 1:
-            import torch.distributed as dist
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(e0.elapsed_time(e1) / steps, ws, dev)
 
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
     ms_max = timed(run, args.steps)
     clk = clocks.stop()
-    value = ws * packed_bytes / (ms_max * 1e-3) / 1e9
+    value = whole_job_gbs(ws, packed_bytes, ms_max)
     ms_chain = timed(run_chain, args.steps)
-    chain_val = ws * packed_bytes / (ms_chain * 1e-3) / 1e9
+    chain_val = whole_job_gbs(ws, packed_bytes, ms_chain)
 
     # end to end through the public API: pinned host x in, host y out
     xh = torch.empty(prob.xdev.shape, dtype=prob.xdev.dtype, pin_memory=True)
@@ -388,7 +400,7 @@ def run_ours(args, w, M):
         yh.copy_(prob.ydev, non_blocking=True)
 
     ms_e2e = timed(e2e_step, args.steps)
-    e2e_val = ws * packed_bytes / (ms_e2e * 1e-3) / 1e9
+    e2e_val = whole_job_gbs(ws, packed_bytes, ms_e2e)
     launches = prob.kernel_launches
     hbm, src = peaks()
     tc_peak, tc_src = tensor_peak()

@@ -434,12 +434,12 @@ def run_ours(args, w, M):
 
     configs, variants = {}, {}
     if not args.quick:
-        for wi, w2 in enumerate(wl.WORKLOADS):
+        for w2 in wl.WORKLOADS:
             Ms = [m for m in w2.Ms if not (w2 is w and m == M)]
             if not Ms:
                 continue
             mats2 = mats if w2 is w else pack_workload(w2, dev)
-            configs[f"config{wi + 1}"] = measure(w2, mats2, Ms)
+            configs[w2.name.split(" ")[0]] = measure(w2, mats2, Ms)
             if w2 is not w:
                 del mats2
                 torch.cuda.empty_cache()

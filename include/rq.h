@@ -21,7 +21,8 @@
  *
  * Conventions shared by every call:
  *   - W is stored [N][K] row-major (row n = output feature, K = input
- *     features); groups run along K. x is bf16 [M][K], y is fp32 [M][N].
+ *     features); groups run along K. x is bf16 [M][K], y is fp32 [M][N]
+ *     (or bf16 with rq_wgemm_out / rq_wgemm_batch_out).
  *   - Every pointer named "device" is CUDA device memory that the CALLER
  *     allocated and owns; the library allocates nothing and keeps no state
  *     between calls. Every such pointer must be 16-byte aligned.
@@ -220,8 +221,10 @@ typedef enum rq_out_type {
 /* rq_wgemm / rq_wgemm_batch with the output element type chosen: y is fp32
  * [M][N] (RQ_OUT_F32) or bf16 [M][N] (RQ_OUT_BF16). The bf16 result is
  * exactly the RQ_OUT_F32 result rounded to nearest even, written by the same
- * launch (no second pass over y): the bf16-output epilogue of the batched
- * r/k/v launch ([rwkv_quant_nv] "Operator Optimization Details"). Same
+ * launch (no second pass over y), so a batched r/k/v launch
+ * ([rwkv_quant_nv] "Operator Optimization Details": r/k/v in one kernel) can
+ * hand its outputs on in the bf16 that every product here takes as x (the
+ * pages give no output type; this one is this library's choice). Same
  * validation and ordering rules as rq_wgemm; any other out_type is
  * RQ_ERR_INVALID_ARG. */
 int rq_wgemm_out(const void *x, int M, int K, int N, const rq_packed *w, void *y, int out_type, void *stream);

@@ -8,12 +8,17 @@
  * What it computes, step by step, in plain loops:
  *   - symmetric group quantization (RTN, or a grid search weighted by the
  *     per-channel mean square of the input activation, E[x^2]) into the int4
- *     group-64 and int8 group-16 formats;
- *   - the asymmetric int4 superblock format (groups of 32, eight groups per
- *     superblock, 6-bit group scale and min against fp16 superblock scale/min);
+ *     group-64, int8 group-16 / group-64 and 6-bit group-16 formats;
+ *   - the asymmetric 4-, 5- and 6-bit superblock formats (groups of 32, eight
+ *     groups per superblock, 6-bit group scale and min against fp16
+ *     superblock scale/min);
  *   - exact fp32 dequantization of every format;
  *   - the product y[m][n] = sum_k x[m][k] * w_hat[n][k], summed in fp64 in
- *     ascending k.
+ *     ascending k;
+ *   - the activation statistic E[x^2] in a fixed fp64 summation order;
+ *   - GPTQ on the preset's grid: the input Hessian and the column loop with
+ *     error feedback into every format (the factor U of the damped inverse
+ *     Hessian is computed in oracle/__init__.py with numpy's LAPACK steps).
  *
  * Sources (web pages; cited by title and section):
  *   [ART]  "rwkv-quant: keeping one matrix in bf16 removes 39% of RWKV-7 2.9B's
@@ -26,7 +31,8 @@
  *          "Format & loading": group-wise (group 64) symmetric int4 weights
  *          stored as a code tensor plus a scale tensor; summary paragraph:
  *          kernel output is bit-identical to the offline dequantization, and
- *          calibration-free RTN is the baseline.
+ *          calibration-free RTN is the baseline; section "Accuracy warning":
+ *          the int8 w8g64 tier.
  *
  * Where the pages leave a step open the plainest reading is taken; every such
  * reading is listed in the design notes and restated at the function below.

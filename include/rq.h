@@ -231,9 +231,13 @@ int rq_wgemm_out(const void *x, int M, int K, int N, const rq_packed *w, void *y
 int rq_wgemm_batch_out(const rq_wgemm_item *items, int count, int M, int out_type, void *stream);
 
 /* Export w_hat as fp32 [N][K] into W_out (device).  ([CARD] summary: the
- * kernel output is bit-identical to the offline dequantization.) Uses the
- * same device unpack as rq_wgemm; bit-exact: q * scale for the symmetric
- * formats, fp32(S_j * q - M_j) for the superblock formats. */
+ * kernel output is bit-identical to the offline dequantization.) Bit-exact:
+ * q * scale for the symmetric formats, fp32(S_j * q - M_j) for the
+ * superblock formats, the values the oracle's dequantization gives. The
+ * products do not go through this export: rq_wgemm unpacks the same codes
+ * with its own in-register arithmetic (see there for its rounding), so its
+ * outputs agree with x * (this w_hat)^T within the stated tolerance, and
+ * exactly whenever every partial sum is exact (integer-valued cases). */
 int rq_dequant(const rq_packed *w, float *W_out, void *stream);
 
 /* Accumulate the statistic of the E[x^2]-weighted search on the device.
@@ -244,12 +248,15 @@ int rq_dequant(const rq_packed *w, float *W_out, void *stream);
  *   sum_sq  device fp64 [K], caller-owned running sums: the call adds
  *           sum_r x[r][k]^2 to sum_sq[k]. Zero it before the first batch;
  *           call once per batch of rows.
- * Summation order (deterministic, bit-reproducible): the R rows are cut into
- * 64 contiguous chunks of ceil(R / 64) rows (the last ones may be short or
- * empty); each chunk is summed in fp64 in ascending row order starting from
- * 0, the 64 chunk sums are added in ascending chunk order starting from 0,
- * and that total is added to sum_sq[k]. Squares of bf16 values are exact in
- * fp64. Limits: 1 <= R <= 2^24, 1 <= K <= 2^20. Non-finite x: unspecified. */
+ * The statistic is the mean of x_k^2 over all calibration rows; the pages fix
+ * no summation order. Squares of bf16 values are exact in fp64, so the result
+ * differs from one ascending fp64 sum over the rows only by the rounding of
+ * the additions: |difference| <= 2 (R + 1) 2^-53 sum_sq[k] (and none at all
+ * when every partial sum is exact, e.g. for activations that are small
+ * multiples of a common power of two). The device order is fixed (each CTA
+ * sums interleaved rows ascending, then its row phases and the CTAs of a
+ * cluster in order), so repeated calls give the same bits.
+ * Limits: 1 <= R <= 2^24, 1 <= K <= 2^20. Non-finite x: unspecified. */
 int rq_act_sumsq(const void *x, int R, int K, double *sum_sq, void *stream);
 
 /* act_sq[k] = fp32(sum_sq[k] / rows) (one fp64 division, one rounding to
@@ -317,6 +324,19 @@ int rq_last_cuda_error(void);
  * RQ_ERR_DEVICE_TIMEOUT if a wait bit was set, RQ_ERR_NOT_POSITIVE_DEFINITE
  * if only the pivot bit was, or RQ_ERR_CUDA. */
 int rq_device_status(void *stream, int *word);
+
+/* Testing hook for the bounded device waits (the pages have no counterpart;
+ * this exists so that the give-up paths can be exercised without a fault).
+ * Every later launch from any host thread uses:
+ *   wait_ns  the bound of each device wait, in nanoseconds; 0 restores the
+ *            default of 2 s. At most 60 s.
+ *   flags    bit 0 (1): the threads that issue the weight copies of the
+ *            products issue none, so every wait for a copy runs out after
+ *            wait_ns; the call then completes with unspecified y and
+ *            rq_device_status reports RQ_ERR_DEVICE_TIMEOUT. 0 = normal.
+ * Returns RQ_ERR_INVALID_ARG for other values. Not for production use: set
+ * it back with rq_test_hooks(0, 0). */
+int rq_test_hooks(long long wait_ns, int flags);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int rq_version(void);

@@ -265,9 +265,9 @@ def wgemm(fmt: str, x_bf16_bits, K: int, N: int, codes, scales, rows=None) -> np
 
 def act_sumsq(x_bf16_bits, sum_sq=None) -> np.ndarray:
     """Running per-channel sums of x^2 over the rows of x (raw bf16 bits,
-    uint16 [R][K]) added into ``sum_sq`` (fp64 [K], zeros when None), in the
-    order of the design notes: 64 contiguous row chunks, each summed ascending,
-    then the chunk sums ascending."""
+    uint16 [R][K]) added into ``sum_sq`` (fp64 [K], zeros when None): each
+    channel's squares are added to its running sum one row at a time, rows
+    ascending, in fp64."""
     x = _c(x_bf16_bits, np.uint16)
     R, K = x.shape
     out = np.zeros(K, dtype=np.float64) if sum_sq is None else np.array(sum_sq, dtype=np.float64, copy=True)

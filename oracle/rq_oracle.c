@@ -676,28 +676,20 @@ void orc_wgemm(int fmt, const uint16_t *x, int M, int K, int N, const uint8_t *c
 /* ------------------------------------------------------------------------ */
 
 /* [ART] "Two presets and six sizes": the search weights input channel k by
- * E[x_k^2], the mean over calibration rows of the squared activation. The
- * pages fix no summation order; the reading here (the same for the device
- * call) is: cut the R rows into 64 contiguous chunks of ceil(R / 64) rows,
- * sum each chunk in fp64 in ascending row order starting from 0, add the 64
- * chunk sums in ascending order starting from 0, and add that total to the
- * running sum of channel k. x[r][k]^2 of a bf16 value is exact in fp64. */
+ * E[x_k^2], the mean over the calibration rows of the squared activation.
+ * Written as that definition: for each channel the square of every row is
+ * added to the channel's running sum, one row at a time in ascending row
+ * order, in fp64 (x[r][k]^2 of a bf16 value is exact in fp64). A batch of
+ * rows continues the sum of the batches before it. */
 void orc_act_sumsq(const uint16_t *x, int R, int K, double *sum_sq)
 {
-    int rc = (R + 63) / 64;
     for (int k = 0; k < K; k++) {
-        double total = 0.0;
-        for (int c = 0; c < 64; c++) {
-            int r0 = c * rc < R ? c * rc : R;
-            int r1 = r0 + rc < R ? r0 + rc : R;
-            double part = 0.0;
-            for (int r = r0; r < r1; r++) {
-                double v = (double)orc_bf16_to_f32(x[(size_t)r * K + k]);
-                part = part + v * v;
-            }
-            total = total + part;
+        double s = sum_sq[k];
+        for (int r = 0; r < R; r++) {
+            double v = (double)orc_bf16_to_f32(x[(size_t)r * K + k]);
+            s = s + v * v;
         }
-        sum_sq[k] = sum_sq[k] + total;
+        sum_sq[k] = s;
     }
 }
 

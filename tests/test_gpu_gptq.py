@@ -74,7 +74,7 @@ def test_prepare_matches_oracle(K, dead_ch):
         x[:, dead_ch] = 0
     Hd = rq.rq_hessian_accum(x.cuda())
     U, dead = rq.rq_gptq_prepare(Hd, 0.01)
-    Ur, deadr = oracle.gptq_prepare(Hd.cpu().numpy(), 0.01)
+    Ur, deadr = oracle.gptq_prepare(oracle.hessian_accum(wl.bf16_bits(x)), 0.01)
     Ug = U.cpu().numpy()
     assert np.array_equal(dead.cpu().numpy(), deadr)
     assert np.count_nonzero(np.tril(Ug, -1)) == 0
@@ -152,8 +152,7 @@ def test_gptq_full_width_sampled_rows():
     rows against the oracle given the same U."""
     K, N, R = 2048, 2048, 4096
     x = calib_x(130, R, K, rank=256)
-    H = rq.rq_hessian_accum(x.cuda())
-    Hn = H.cpu().numpy()
+    Hn = oracle.hessian_accum(wl.bf16_bits(x))
     Ur, deadr = oracle.gptq_prepare(Hn)
     W = wl.random_matrix(131, N, K)
     p = rq.rq_gptq_quantize_pack(W.cuda(), "w4g64", to_dev(Ur), to_dev(deadr), None, 64)

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import headroom
 import oracle
 import weight_only_quantized_rq_b200 as rq
 from weight_only_quantized_rq_b200 import workloads as wl
@@ -67,14 +68,7 @@ def make_x(seed, M, K, a=None):
     return x, wl.bf16_bits(x)
 
 
-def check_y(y, y_ref, xbits, w_hat, rel=5e-3, elem=1e-2):
-    xf = (xbits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    bound = elem * (np.abs(xf) @ np.abs(w_hat.astype(np.float64)).T)
-    err = np.abs(y.astype(np.float64) - y_ref)
-    nrm = np.linalg.norm(y_ref)
-    assert np.linalg.norm(err) <= rel * max(nrm, 1e-30), (np.linalg.norm(err) / nrm)
-    bad = err > bound + 1e-30
-    assert not bad.any(), f"{bad.sum()} elements outside 1e-2*sum|x||w|"
+check_y = headroom.check_y
 
 
 # --------------------------------------------------------- quantize-pack ---
@@ -225,7 +219,7 @@ def test_wgemm_matches_oracle(case):
     x, xb = make_x(500 + case, M, K, a)
     y = rq.rq_wgemm(x.cuda(), p).cpu().numpy()
     y_ref = oracle.wgemm(fmt, xb, K, N, oc, osc)
-    check_y(y, y_ref, xb, oracle.dequant(fmt, K, N, oc, osc))
+    check_y(y, y_ref, xb, oracle.dequant(fmt, K, N, oc, osc), fmt)
 
 
 @pytest.mark.parametrize("fmt,unit", [("w4g64", 2.0 ** -6), ("w8g16", 2.0 ** -10)])
@@ -307,7 +301,7 @@ def _full_size_check(widx, layer_sample=1, rows_per_matrix=48, Ms=None):
             xb = wl.bf16_bits(x)
             y = rq.rq_wgemm(x.cuda(), p).cpu().numpy()
             y_ref = oracle.wgemm(m.fmt, xb, m.K, len(rows), oc, osc)
-            check_y(y[:, rows], y_ref, xb, oracle.dequant(m.fmt, m.K, len(rows), oc, osc))
+            check_y(y[:, rows], y_ref, xb, oracle.dequant(m.fmt, m.K, len(rows), oc, osc), m.fmt)
         del p
 
 
@@ -347,7 +341,7 @@ def test_wgemm_batch_matches_oracle(fmt, shapes, M):
     rq.rq_wgemm_batch(xs, ws, ys)
     torch.cuda.synchronize()
     for y, (y_ref, xb, wd), (big, n) in zip(ys, refs, bigs):
-        check_y(y.cpu().numpy(), y_ref, xb, wd)
+        check_y(y.cpu().numpy(), y_ref, xb, wd, fmt)
         assert bool(torch.isnan(big[:256]).all()) and bool(torch.isnan(big[256 + n:]).all())
 
 

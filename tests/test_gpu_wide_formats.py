@@ -16,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import headroom
 import oracle
 import weight_only_quantized_rq_b200 as rq
 from weight_only_quantized_rq_b200 import workloads as wl
@@ -59,14 +60,7 @@ def gpu_scales(p, K, N, fmt):
     return raw[:used].view(np.uint16).reshape(N, -1)
 
 
-def check_y(y, y_ref, xbits, w_hat, rel=5e-3, elem=1e-2):
-    xf = (xbits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    bound = elem * (np.abs(xf) @ np.abs(w_hat.astype(np.float64)).T)
-    err = np.abs(y.astype(np.float64) - y_ref)
-    nrm = np.linalg.norm(y_ref)
-    assert np.linalg.norm(err) <= rel * max(nrm, 1e-30), (np.linalg.norm(err) / nrm)
-    bad = err > bound + 1e-30
-    assert not bad.any(), f"{bad.sum()} elements outside 1e-2*sum|x||w|"
+check_y = headroom.check_y
 
 
 def weights_for(seed, N, K, outliers):
@@ -173,7 +167,7 @@ def test_wgemm_matches_oracle(fmt, case):
     x = wl.random_x(1500 + case, M, K, a)
     xb = wl.bf16_bits(x)
     y = rq.rq_wgemm(x.cuda(), p).cpu().numpy()
-    check_y(y, oracle.wgemm(fmt, xb, K, N, oc, None), xb, oracle.dequant(fmt, K, N, oc, None))
+    check_y(y, oracle.wgemm(fmt, xb, K, N, oc, None), xb, oracle.dequant(fmt, K, N, oc, None), fmt)
 
 
 @pytest.mark.parametrize("fmt,shapes,M", [
@@ -197,7 +191,7 @@ def test_wgemm_batch_matches_oracle(fmt, shapes, M):
     rq.rq_wgemm_batch(xs, ws, ys)
     torch.cuda.synchronize()
     for y, (y_ref, xb, wd), (big, n) in zip(ys, refs, bigs):
-        check_y(y.cpu().numpy(), y_ref, xb, wd)
+        check_y(y.cpu().numpy(), y_ref, xb, wd, fmt)
         assert bool(torch.isnan(big[:256]).all()) and bool(torch.isnan(big[256 + n:]).all())
 
 
@@ -219,7 +213,7 @@ def test_full_size_head_sampled(fmt):
         xb = wl.bf16_bits(x)
         y = rq.rq_wgemm(x.cuda(), p).cpu().numpy()
         check_y(y[:, rows], oracle.wgemm(fmt, xb, K, len(rows), oc, None), xb,
-                oracle.dequant(fmt, K, len(rows), oc, None))
+                oracle.dequant(fmt, K, len(rows), oc, None), fmt)
 
 
 # --------------------------------------- symmetric 6-bit g16 and int8 g64 ---
@@ -273,7 +267,7 @@ def test_sym_wgemm_matches_oracle(fmt, case):
     x = wl.random_x(2500 + case, M, K, a)
     xb = wl.bf16_bits(x)
     y = rq.rq_wgemm(x.cuda(), p).cpu().numpy()
-    check_y(y, oracle.wgemm(fmt, xb, K, N, oc, osc), xb, oracle.dequant(fmt, K, N, oc, osc))
+    check_y(y, oracle.wgemm(fmt, xb, K, N, oc, osc), xb, oracle.dequant(fmt, K, N, oc, osc), fmt)
 
 
 @pytest.mark.parametrize("M", [1, 2])
@@ -311,4 +305,4 @@ def test_sym_wgemm_batch_matches_oracle(fmt, shapes, M):
     rq.rq_wgemm_batch(xs, ws, ys)
     torch.cuda.synchronize()
     for y, (y_ref, xb, wd) in zip(ys, refs):
-        check_y(y.cpu().numpy(), y_ref, xb, wd)
+        check_y(y.cpu().numpy(), y_ref, xb, wd, fmt)

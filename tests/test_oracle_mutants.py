@@ -55,10 +55,10 @@ MUTANTS = [
     ("GPTQ superblock error without the min", "double err = (w[k] - (double)asym_deq(q, Sj, Mj)) / U[(size_t)k * K + k];",
      "double err = (w[k] - (double)((float)q * Sj)) / U[(size_t)k * K + k];", None),
     ("Hessian skips the last row", "for (int r = 0; r < R; r++) {\n                double xi", "for (int r = 0; r < R - 1; r++) {\n                double xi", None),
-    ("E[x^2] sums |x| instead of x^2", "part = part + v * v;", "part = part + fabs(v);", None),
-    ("E[x^2] skips the last chunk", "for (int c = 0; c < 64; c++) {\n            int r0", "for (int c = 0; c < 63; c++) {\n            int r0", None),
+    ("E[x^2] sums |x| instead of x^2", "s = s + v * v;", "s = s + fabs(v);", None),
+    ("E[x^2] skips the last row", "for (int r = 0; r < R; r++) {\n            double v", "for (int r = 0; r < R - 1; r++) {\n            double v", None),
     ("E[x^2] divides by rows - 1", "act_sq[k] = (float)(sum_sq[k] / (double)rows);", "act_sq[k] = (float)(sum_sq[k] / (double)(rows - 1));", None),
-    ("E[x^2] overwrites the running sum", "sum_sq[k] = sum_sq[k] + total;", "sum_sq[k] = total;", None),
+    ("E[x^2] drops the running sum", "double s = sum_sq[k];", "double s = 0.0;", None),
 ]
 
 

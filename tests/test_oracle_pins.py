@@ -553,7 +553,7 @@ def test_act_stats_integer_rows_exact(orc):
     """Small-integer activations: every partial sum is an exact integer in
     fp64, so the result is the integer sum of squares over R, rounded once."""
     rng = np.random.default_rng(31)
-    R, K = 4097, 67           # 64 chunks of 65 rows: the last chunk holds 2 rows
+    R, K = 4097, 67
     xi = rng.integers(-40, 41, size=(R, K))
     s = orc.act_sumsq(_bf16_bits(xi.astype(np.float32)))
     assert np.array_equal(s, (xi.astype(np.int64) ** 2).sum(0).astype(np.float64))

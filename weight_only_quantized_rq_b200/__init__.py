@@ -50,7 +50,7 @@ SB_FORMATS = (RQ_W4_ASYM_SB32, RQ_W5_ASYM_SB32, RQ_W6_ASYM_SB32)
 EXPORTS = ("rq_packed_size", "rq_quantize_pack", "rq_wgemm", "rq_wgemm_batch", "rq_wgemm_out", "rq_wgemm_batch_out",
            "rq_dequant",
            "rq_act_sumsq", "rq_act_finalize", "rq_hessian_accum", "rq_gptq_prepare", "rq_gptq_quantize_pack",
-           "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_version")
+           "rq_status_string", "rq_last_cuda_error", "rq_device_status", "rq_test_hooks", "rq_version")
 MAX_BATCH = 160
 TC_MIN_M = 3         # activation rows from which int4/int8/4-bit superblock products run on the tensor cores
                      # (5- and 6-bit products run there at every M)
@@ -131,6 +131,8 @@ def _lib() -> ctypes.CDLL:
         L.rq_last_cuda_error.restype = I
         L.rq_device_status.argtypes = [P, ctypes.POINTER(I)]
         L.rq_device_status.restype = I
+        L.rq_test_hooks.argtypes = [ctypes.c_longlong, I]
+        L.rq_test_hooks.restype = I
         L.rq_version.argtypes = []
         L.rq_version.restype = I
         _L = L
@@ -347,6 +349,12 @@ def rq_device_status(stream=None) -> int:
     if st not in (RQ_OK, RQ_ERR_DEVICE_TIMEOUT, RQ_ERR_NOT_POSITIVE_DEFINITE):
         raise RqError(st, "rq_device_status")
     return word.value
+
+
+def rq_test_hooks(wait_ns: int = 0, flags: int = 0) -> None:
+    """Testing hook: the bound of every device wait (0 = the default 2 s)
+    and flags (1 = issue no weight copies, so the waits run out)."""
+    _check(_lib().rq_test_hooks(int(wait_ns), int(flags)), "rq_test_hooks")
 
 
 # short aliases

@@ -53,6 +53,14 @@ int cuda_status(cudaError_t e) {
 
 namespace rq {
 
+namespace {
+unsigned long long g_wait_ns = 2000000000ull;
+int g_test_flags = 0;
+}  // namespace
+
+unsigned long long wait_limit_ns() { return __atomic_load_n(&g_wait_ns, __ATOMIC_RELAXED); }
+int test_flags() { return __atomic_load_n(&g_test_flags, __ATOMIC_RELAXED); }
+
 int sm_count() {
     static int cache[64] = {0};
     int dev = 0;
@@ -225,6 +233,13 @@ int rq_device_status(void* stream, int* word) {
     return w ? RQ_ERR_NOT_POSITIVE_DEFINITE : RQ_OK;
 }
 
-int rq_version(void) { return 100; }
+int rq_test_hooks(long long wait_ns, int flags) {
+    if (wait_ns < 0 || wait_ns > 60000000000ll || (flags & ~rq::kTestNoCopies) != 0) return RQ_ERR_INVALID_ARG;
+    __atomic_store_n(&rq::g_wait_ns, wait_ns == 0 ? 2000000000ull : (unsigned long long)wait_ns, __ATOMIC_RELAXED);
+    __atomic_store_n(&rq::g_test_flags, flags, __ATOMIC_RELAXED);
+    return RQ_OK;
+}
+
+int rq_version(void) { return 200; }
 
 }  // extern "C"

@@ -2,11 +2,11 @@
 // inline-PTX wrappers (mbarrier, bulk async copy, programmatic dependent
 // launch), bounded waits, and the in-register unpack of packed codes.
 //
-// The unpack functions are the single definition of how a stored code becomes
-// a number; rq_dequant and the GEMV both use them, so the exported w_hat and
-// the w_hat inside the product are the same values ("kernel output is
-// bit-identical to the offline dequant": RWKV-7 G1 1.5B int4 model card,
-// summary paragraph).
+// Each unpack below turns stored codes into exact numbers (128 + u, 1024 + u,
+// q); the kernels then apply the scales in their own arithmetic: rq_dequant
+// forms w_hat = q * s exactly (the offline dequantization, RWKV-7 G1 1.5B
+// int4 model card, summary paragraph), the products fold the scale into fp32
+// sums, and agree with x * w_hat^T within the library's stated tolerance.
 #pragma once
 
 #include <cstdint>
@@ -37,7 +37,8 @@ __device__ __forceinline__ void store_y(void* y, size_t idx, float v, int bf16) 
 // needed); each kernel file exports a host accessor that reads and clears it.
 static __device__ unsigned g_status = 0u;
 
-// Wall-clock bound of every device spin-wait, in nanoseconds.
+// Default wall-clock bound of a device spin-wait, in nanoseconds (launches
+// pass the bound they were given, which is this unless a test changed it).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -98,17 +99,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // critical path (a producer waiting for a free slot), so that polling does
 // not take issue slots from the warps that compute.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned flag,
-                                                  unsigned nap_ns = 0u) {
+                                                  unsigned nap_ns = 0u,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (nap_ns) __nanosleep(nap_ns);
         if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
-        if ((it & 15u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((it & 15u) == 0u && globaltimer_ns() - t0 > limit_ns) {
             atomicOr(&g_status, flag);
             return false;
         }
     }
+}
+
+// Named barrier of n threads (id 1..15) that ANDs a flag over them: threads
+// that give up on a wait still take part, so every participant learns of it
+// and none is left waiting at the barrier.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+                 : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(n) : "memory");
+    return r != 0;
 }
 
 // ------------------------------------------------------ bulk async copy ---
@@ -140,19 +152,6 @@ __device__ __forceinline__ void grid_dep_launch() {
 }
 
 // ------------------------------------------------------------- loads ------
-__device__ __forceinline__ uint4 lds128(const void* p) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
-    return v;
-}
-__device__ __forceinline__ float4 lds128f(const void* p) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(smem_u32(p)));
-    return v;
-}
-
 // Loads from 32-bit shared-memory addresses (no generic-to-shared conversion
 // per access). Volatile keeps them after the barrier waits that guard them.
 __device__ __forceinline__ uint4 lds128_a(uint32_t a) {
@@ -180,12 +179,6 @@ __device__ __forceinline__ uint32_t lds16_a(uint32_t a) {
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
     return v;
 }
-__device__ __forceinline__ float ldsf_a(uint32_t a) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
-    return v;
-}
-
 // --------------------------------------------------------------- unpack ---
 // int4 codes. A 32-bit word holds eight nibbles; nibble p (bits 4p..4p+3)
 // is the code of weight k = 8i + p of that word (byte j: k = 2j low, 2j+1
@@ -216,9 +209,6 @@ __device__ __forceinline__ void unpack_w4(uint32_t w, float f[8]) {
     f[6] = __uint_as_float(prmt(hi, kW4Magic, 0x7244u));
     f[7] = __uint_as_float(prmt(hi, kW4Magic, 0x7344u));
 }
-// Position inside the word of output slot j of unpack_w4.
-__host__ __device__ constexpr int w4_slot_nibble(int j) { return j < 4 ? 2 * j : 2 * (j - 4) + 1; }
-
 // int4 codes as bf16 pairs (the GEMV and dequant unpack). Pair j (0..3) of a
 // word holds nibble j in its low half and nibble j+4 in its high half, each
 // as the bf16 value 128 + u: the nibble lands in mantissa bits 0..3 under the
@@ -238,27 +228,6 @@ __device__ __forceinline__ uint32_t w4_pair(uint32_t w) {
 __device__ __forceinline__ float bf16lo_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// c + a.half(AH) * b.half(BH), with bf16 operands and an fp32 accumulator:
-// the product of two bf16 values is exact in fp32, so this equals an fp32
-// fma of the two values widened to fp32 (one rounding).
-template <int AH, int BH>
-__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
-    float d;
-    if (AH == 0 && BH == 0)
-        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
-            " fma.rn.f32.bf16 %0, a0, b0, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    else if (AH == 1 && BH == 0)
-        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
-            " fma.rn.f32.bf16 %0, a1, b0, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    else if (AH == 0 && BH == 1)
-        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
-            " fma.rn.f32.bf16 %0, a0, b1, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    else
-        asm("{ .reg .b16 a0, a1, b0, b1; mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;"
-            " fma.rn.f32.bf16 %0, a1, b1, %3; }" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    return d;
-}
-
 // The eight values 128 + u_k of one code word, in natural k order, widened
 // exactly from the bf16 pairs the GEMV multiplies (rq_dequant's unpack).
 __device__ __forceinline__ void w4_word_values(uint32_t w, float o[8]) {
@@ -267,45 +236,6 @@ __device__ __forceinline__ void w4_word_values(uint32_t w, float o[8]) {
     o[1] = bf16lo_f32(r1); o[5] = bf16hi_f32(r1);
     o[2] = bf16lo_f32(r2); o[6] = bf16hi_f32(r2);
     o[3] = bf16lo_f32(r3); o[7] = bf16hi_f32(r3);
-}
-
-// acc[0..NA-1] += the 8 products (128 + u_k) * x_k of one code word, spread
-// over NA independent accumulators (NA = 8: one per position, no chain
-// inside a word; NA = 4 or 2: products folded pairwise).
-template <int NA>
-__device__ __forceinline__ void dot8_w4_split(uint32_t w, uint4 X, float (&acc)[NA]) {
-    const uint32_t r0 = w4_pair<0>(w), r1 = w4_pair<1>(w), r2 = w4_pair<2>(w), r3 = w4_pair<3>(w);
-    acc[0 % NA] = fma_bf16<0, 0>(r0, X.x, acc[0 % NA]);   // u0 x0
-    acc[1 % NA] = fma_bf16<1, 0>(r0, X.z, acc[1 % NA]);   // u4 x4
-    acc[2 % NA] = fma_bf16<0, 1>(r1, X.x, acc[2 % NA]);   // u1 x1
-    acc[3 % NA] = fma_bf16<1, 1>(r1, X.z, acc[3 % NA]);   // u5 x5
-    acc[4 % NA] = fma_bf16<0, 0>(r2, X.y, acc[4 % NA]);   // u2 x2
-    acc[5 % NA] = fma_bf16<1, 0>(r2, X.w, acc[5 % NA]);   // u6 x6
-    acc[6 % NA] = fma_bf16<0, 1>(r3, X.y, acc[6 % NA]);   // u3 x3
-    acc[7 % NA] = fma_bf16<1, 1>(r3, X.w, acc[7 % NA]);   // u7 x7
-}
-
-template <int NA>
-__device__ __forceinline__ float sum_acc(const float (&a)[NA]) {
-    if (NA == 8) return ((a[0 % NA] + a[1 % NA]) + (a[2 % NA] + a[3 % NA])) + ((a[4 % NA] + a[5 % NA]) + (a[6 % NA] + a[7 % NA]));
-    if (NA == 4) return (a[0 % NA] + a[1 % NA]) + (a[2 % NA] + a[3 % NA]);
-    if (NA == 2) return a[0] + a[1 % NA];
-    return a[0];
-}
-
-// acc += sum over the 8 weights of one code word of (128 + u_k) * x_k, where
-// X0..X3 hold x_0..x_7 as natural-order bf16 pairs ((x0,x1), (x2,x3), ...).
-__device__ __forceinline__ float dot8_w4(uint32_t w, uint4 X, float acc) {
-    const uint32_t r0 = w4_pair<0>(w), r1 = w4_pair<1>(w), r2 = w4_pair<2>(w), r3 = w4_pair<3>(w);
-    acc = fma_bf16<0, 0>(r0, X.x, acc);   // u0 x0
-    acc = fma_bf16<1, 0>(r0, X.z, acc);   // u4 x4
-    acc = fma_bf16<0, 1>(r1, X.x, acc);   // u1 x1
-    acc = fma_bf16<1, 1>(r1, X.z, acc);   // u5 x5
-    acc = fma_bf16<0, 0>(r2, X.y, acc);   // u2 x2
-    acc = fma_bf16<1, 0>(r2, X.w, acc);   // u6 x6
-    acc = fma_bf16<0, 1>(r3, X.y, acc);   // u3 x3
-    acc = fma_bf16<1, 1>(r3, X.w, acc);   // u7 x7
-    return acc;
 }
 
 // int4 codes as fp16 pairs (the GEMV unpack). An fp16 mantissa has ten bits,

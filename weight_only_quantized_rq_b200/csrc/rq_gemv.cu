@@ -39,25 +39,14 @@
 #include "rq_device.cuh"
 #include "rq_internal.h"
 
-// Phase marks for external profiling builds; no code in this library.
-#ifndef RQ_PHASE_MARK
-#define RQ_PHASE_MARK(i)
-#endif
-
 namespace rq {
 namespace {
 
-#ifndef RQ_GEMV_WARPS
-#define RQ_GEMV_WARPS 8
-#endif
-constexpr int kConsumerWarps = RQ_GEMV_WARPS;
+constexpr int kConsumerWarps = 8;
 constexpr int kProducerWarp = kConsumerWarps;         // issues the weight copies
 constexpr int kStagerWarp = kConsumerWarps + 1;       // stages x
 constexpr int kThreads = (kConsumerWarps + 2) * 32;
-#ifndef RQ_PRODUCER_NAP_NS
-#define RQ_PRODUCER_NAP_NS 256
-#endif
-constexpr unsigned kProducerNapNs = RQ_PRODUCER_NAP_NS;   // poll interval of the producer's slot waits
+constexpr unsigned kProducerNapNs = 256;                  // poll interval of the producer's slot waits
 constexpr unsigned kStagerNapNs = 512;                   // and of the x stager's buffer waits
 
 struct Item {                  // one product of a launch
@@ -86,6 +75,8 @@ struct Batch {
     uint32_t x_off, x_bytes;   // nxb staged-x buffers (x, then its metadata)
     uint32_t red_off, red_bytes;  // per stage: k-slice partial sums
     uint32_t bar_off;          // full[stages], empty[stages], xfull[2], xempty[2]
+    unsigned long long wait_ns;  // bound of every device wait
+    int test_flags;            // kTestNoCopies: the producer issues no copies (tests the waits)
     Item it[MAXI];
 };
 
@@ -497,6 +488,7 @@ struct Ring {
     int stages;
     int s;                     // stage of the next group
     uint32_t ph;               // its phase parity
+    unsigned long long lim;    // wait bound
 };
 
 // All groups of rows [ra, rb) of item `it` for this warp: waits for each
@@ -515,19 +507,24 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
     const int wfirst = wteam * RW;                       // first row of this warp in a group
     for (int g0 = ra; g0 < rb; g0 += Rg) {
         const int s = ring.s;
-        if (!mbar_wait_bounded(&ring.full[s], ring.ph, kStatusTmaWait)) return false;
+        const bool got = mbar_wait_bounded(&ring.full[s], ring.ph, kStatusTmaWait, 0u, ring.lim);
         if (++ring.s == ring.stages) {                   // next stage and its phase parity
             ring.s = 0;
             ring.ph ^= 1u;
         }
         const int rg = min(Rg, rb - g0);
+        bool all = got;
         if (wfirst < rg) {                               // warp-uniform
             float* red = reinterpret_cast<float*>(ring.red + (size_t)s * ring.red_bytes);
-            gemv_group<FMT, MT, RW, TT, YB>(it, ring.base + (uint32_t)s * ring.stage_bytes, g0, rg, x_s, m0, mrows,
-                                        lane, rbase, slice, red);
+            if (got)
+                gemv_group<FMT, MT, RW, TT, YB>(it, ring.base + (uint32_t)s * ring.stage_bytes, g0, rg, x_s, m0,
+                                                mrows, lane, rbase, slice, red);
             if (KS > 1) {
-                asm volatile("bar.sync %0, %1;" :: "r"(1 + team), "r"(KS * 32) : "memory");
-                if (slice == 0 && lane < RW * MT) {
+                // the k-slices of a team meet here; a slice whose wait gave up
+                // makes the whole team give up together (no warp is left at
+                // the barrier)
+                all = bar_and(1 + team, KS * 32, got);
+                if (all && slice == 0 && lane < RW * MT) {
                     const int r = lane / MT, m = lane - r * MT, rr = wfirst + r;
                     if (rr < rg && m < mrows) {
                         const float* q = red + ((size_t)rr * MT + m) * KS;
@@ -538,6 +535,7 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
                 }
             }
         }
+        if (!all) return false;
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);     // stage consumed
     }
@@ -573,12 +571,11 @@ gemv_kernel(const Batch<MAXI> p) {
     }
     __syncthreads();
     grid_dep_launch();
-    RQ_PHASE_MARK(0);
 
     if (warp == kProducerWarp) {                         // weight copies into the ring
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();
-            int gi = 0;
+            int gi = 0, armed = 0;
             bool ok = true;
             for (int i = item_after(p, lo); i < p.count && ok; ++i) {
                 const Item& it = p.it[i];
@@ -590,10 +587,12 @@ gemv_kernel(const Batch<MAXI> p) {
                 for (int g0 = ra; g0 < rb; g0 += it.Rg, ++gi) {
                     const int s = gi % p.stages;
                     if (gi >= p.stages &&
-                        !mbar_wait_bounded(&empty[s], ((gi / p.stages) - 1) & 1, kStatusSlotWait, kProducerNapNs)) {
+                        !mbar_wait_bounded(&empty[s], ((gi / p.stages) - 1) & 1, kStatusSlotWait, kProducerNapNs,
+                                           p.wait_ns)) {
                         ok = false;
                         break;
                     }
+                    if (p.test_flags & kTestNoCopies) continue;
                     const int rg = min(it.Rg, rb - g0);
                     const uint32_t cb = (uint32_t)rg * it.crb;
                     const uint32_t sb = it.srb ? (((uint32_t)rg * it.srb + 15u) & ~15u) : 0u;
@@ -602,7 +601,14 @@ gemv_kernel(const Batch<MAXI> p) {
                     bulk_g2s(st, it.codes + (size_t)g0 * it.crb, cb, &full[s], pol);
                     if (sb)
                         bulk_g2s(st + round16((size_t)it.Rg * it.crb), it.scales + (size_t)g0 * it.srb, sb, &full[s], pol);
+                    armed = gi + 1;
                 }
+            }
+            // Copies still in flight (consumers that gave up) land before the CTA
+            // leaves: wait for the last phase armed on every stage.
+            for (int s = 0; s < p.stages && s < armed; ++s) {
+                const int uses = armed / p.stages + (s < armed % p.stages ? 1 : 0);
+                mbar_wait_bounded(&full[s], (uint32_t)(uses - 1) & 1u, kStatusTmaWait, kProducerNapNs, p.wait_ns);
             }
         }
         return;
@@ -628,7 +634,8 @@ gemv_kernel(const Batch<MAXI> p) {
             item_units(it, lo, hi, ua, ub);
             if (ua * it.rho >= min(ub * it.rho, it.N)) continue;
             const int b = xi % p.nxb;
-            if (xi >= p.nxb && !mbar_wait_bounded(&xempty[b], ((xi / p.nxb) - 1) & 1, kStatusXWait, kStagerNapNs))
+            if (xi >= p.nxb &&
+                !mbar_wait_bounded(&xempty[b], ((xi / p.nxb) - 1) & 1, kStatusXWait, kStagerNapNs, p.wait_ns))
                 break;
             stage_x<FMT, MT>(it, p.m0, p.mrows, smem + p.x_off + (size_t)b * p.x_bytes, lane, 32);
             mbar_arrive(&xfull[b]);                      // each lane: its stores are released
@@ -644,7 +651,6 @@ gemv_kernel(const Batch<MAXI> p) {
         stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, tid, kCoop);
         asm volatile("bar.sync %0, %1;" :: "n"(kCoopBarrier), "n"(kCoop) : "memory");
     }
-    RQ_PHASE_MARK(1);
     Ring ring;
     ring.full = full;
     ring.empty = empty;
@@ -655,6 +661,7 @@ gemv_kernel(const Batch<MAXI> p) {
     ring.stages = p.stages;
     ring.s = 0;
     ring.ph = 0u;
+    ring.lim = p.wait_ns;
     int xi = 0;                                          // items done
     for (int i = i_first < 0 ? p.count : i_first; i < p.count; ++i) {
         const Item it = p.it[i];                         // this item's fields in registers
@@ -665,8 +672,7 @@ gemv_kernel(const Batch<MAXI> p) {
         const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
         if (ra >= rb) continue;
         const int b = xi % p.nxb;
-        if (!mbar_wait_bounded(&xfull[b], (xi / p.nxb) & 1, kStatusXWait)) return;
-        RQ_PHASE_MARK(2);
+        if (!mbar_wait_bounded(&xfull[b], (xi / p.nxb) & 1, kStatusXWait, 0u, p.wait_ns)) return;
         const uint32_t x_s = smem_s + p.x_off + (uint32_t)b * p.x_bytes;
         bool ok;
         if (it.T == 32) {                                // whole-warp teams: the common case
@@ -683,22 +689,14 @@ gemv_kernel(const Batch<MAXI> p) {
         if (lane == 0) mbar_arrive(&xempty[b]);          // staged x released
         ++xi;
     }
-    RQ_PHASE_MARK(4);
 }
 
 // Shared-memory target per CTA for single products: three CTAs (three kernels
 // of a dependent chain) fit on one SM. Batches run two CTAs per SM.
-#ifndef RQ_GEMV_SINGLE_CTAS_PER_SM
-#define RQ_GEMV_SINGLE_CTAS_PER_SM 1
-#endif
-#ifndef RQ_GEMV_BATCH_CTAS_PER_SM
-#define RQ_GEMV_BATCH_CTAS_PER_SM 2
-#endif
+constexpr int kSingleCtasPerSm = 1;
+constexpr int kBatchCtasPerSm = 2;
 constexpr size_t kSmemTarget = 72 * 1024;
-#ifndef RQ_GEMV_SMEM_BATCH_KB
-#define RQ_GEMV_SMEM_BATCH_KB 112
-#endif
-constexpr size_t kSmemBatch = RQ_GEMV_SMEM_BATCH_KB * 1024;
+constexpr size_t kSmemBatch = 112 * 1024;
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemAttr = kSmemLimit + 1024;
 
@@ -754,12 +752,8 @@ Layout layout_of(int fmt, int K) {
 
 // Rows per team for a product: the largest of 4, 2, 1 whose group of
 // teams * RW rows stays within 48 KB.
-#ifndef RQ_GEMV_RW_MAX
-#define RQ_GEMV_RW_MAX 4
-#endif
 int rw_allowed(int fmt, int K) {
     const Layout l = layout_of(fmt, K);
-    if (RQ_GEMV_RW_MAX < 4) return RQ_GEMV_RW_MAX;
     auto sb = [&](size_t R) { return round16(R * code_row_bytes(fmt, K)) + round16(R * scale_row_bytes(fmt, K)); };
     if (sb((size_t)l.teams * 4) <= 48 * 1024) return 4;
     return sb((size_t)l.teams * 2) <= 48 * 1024 ? 2 : 1;
@@ -850,7 +844,9 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
             return cudaErrorInvalidValue;
         }
         p.total = total;
-        int grid = sm_count() * (count > 1 ? RQ_GEMV_BATCH_CTAS_PER_SM : RQ_GEMV_SINGLE_CTAS_PER_SM);
+        p.wait_ns = wait_limit_ns();
+        p.test_flags = test_flags();
+        int grid = sm_count() * (count > 1 ? kBatchCtasPerSm : kSingleCtasPerSm);
         if (count == 1 && grid > units_min) grid = (int)units_min;
         int stages = sp.stages;
         if (count == 1) {   // a single product needs no more stages than its largest CTA has groups

@@ -116,4 +116,12 @@ cudaError_t status_tc(cudaStream_t st, unsigned* word);
 
 int sm_count();   // multiprocessors of the current device
 
+// Bound of every device wait that a launch passes to its kernel (2 s unless
+// rq_test_hooks set another), and the testing flags rq_test_hooks set
+// (bit 0: the threads that issue weight copies issue none, so the waits for
+// them run out).
+unsigned long long wait_limit_ns();
+int test_flags();
+constexpr int kTestNoCopies = 1;
+
 }  // namespace rq

@@ -70,14 +70,6 @@
 #include "rq_device.cuh"
 #include "rq_internal.h"
 
-// Timestamp marks for external profiling builds; no code in this library.
-#ifdef RQ_TC_TRACE_HEADER
-#include RQ_TC_TRACE_HEADER
-#endif
-#ifndef RQ_TC_MARK
-#define RQ_TC_MARK(ev, i)
-#endif
-
 namespace rq {
 namespace {
 
@@ -114,6 +106,8 @@ struct TcArgs {
     int AS;                         // A slots in tensor memory
     uint32_t A0;                    // first tensor-memory column of the A slots (after 2 * niss accumulators)
     uint32_t stage_bytes, x_atom, codes_off, bar_off, tx_bytes;
+    unsigned long long wait_ns;     // bound of every device wait
+    int test_flags;                 // kTestNoCopies: the copy thread issues nothing (tests the waits)
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -450,8 +444,8 @@ __device__ __forceinline__ void dq_w6(const uint4 c, const uint2 pl, uint32_t sc
 // ------------------------------------------------------------ work units
 struct Unit { int item, n0, t0, t1; };
 
-template <int MAXI>
-__device__ __forceinline__ bool get_unit(const TcArgs<MAXI>& p, int i, Unit& u) {
+template <class P>
+__device__ __forceinline__ bool get_unit(const P& p, int i, Unit& u) {
     if (p.split > 1) {                       // one tile, one K range per CTA of the cluster
         if (i > 0) return false;
         const int tile = (int)blockIdx.x / p.split, j = (int)cluster_rank();
@@ -482,9 +476,9 @@ __device__ __forceinline__ bool get_unit(const TcArgs<MAXI>& p, int i, Unit& u) 
 // stage) sequence as every role of the CTA. Per stage a thread takes a
 // quarter of the stage's K: int4 one scale (64 weights at 256-K stages, 32 at
 // 128-K stages), int8 two (32 weights).
-template <int FMT, int KS, int MAXI>
+template <int FMT, int KS, class P>
 struct ScaleCursor {
-    const TcArgs<MAXI>* p;
+    const P* p;
     int ui, t;
     Unit u;
     bool valid;
@@ -501,7 +495,7 @@ struct ScaleCursor {
         groups = it.K / sym_group(FMT);
         t = u.t0;
     }
-    __device__ __forceinline__ void start(const TcArgs<MAXI>* prm, int rr, int hh) {
+    __device__ __forceinline__ void start(const P* prm, int rr, int hh) {
         p = prm;
         r = rr;
         h = hh;
@@ -550,13 +544,14 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // 23 warps per CTA most of them wait most of the time: sleeping waiters leave
 // the issue slots to the warps that dequantize. Gives up after kWaitLimitNs,
 // ORs `flag` into the status word and returns false.
-__device__ __forceinline__ bool nap_wait(uint64_t* bar, uint32_t parity, unsigned flag, unsigned nap_ns) {
+__device__ __forceinline__ bool nap_wait(uint64_t* bar, uint32_t parity, unsigned flag, unsigned nap_ns,
+                                         unsigned long long lim) {
     if (mbar_test(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         __nanosleep(nap_ns);
         if (mbar_test(bar, parity)) return true;
-        if ((it & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((it & 63u) == 0u && globaltimer_ns() - t0 > lim) {
             atomicOr(&g_status, flag);
             return false;
         }
@@ -567,8 +562,9 @@ __device__ __forceinline__ bool nap_wait(uint64_t* bar, uint32_t parity, unsigne
 // nap_ns == 0: waits on the critical path (dequantizing warps, MMA issue) use
 // the suspending try_wait, which measured faster there than sleeping between
 // tests; the long waits (epilogue, drains) sleep.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned flag, unsigned nap_ns) {
-    const bool ok = nap_ns ? nap_wait(bar, parity, flag, nap_ns) : mbar_wait_bounded(bar, parity, flag);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned flag, unsigned nap_ns,
+                                          unsigned long long lim) {
+    const bool ok = nap_ns ? nap_wait(bar, parity, flag, nap_ns, lim) : mbar_wait_bounded(bar, parity, flag, 0u, lim);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -626,7 +622,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tslot;
     grid_dep_launch();
-    if (tid == 0) RQ_TC_MARK(1, 0);
 
     if (warp < 2) {
         // ------------------------------------------------------ MMA issue
@@ -642,7 +637,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             Unit u;
             for (int ui = 0; ok && get_unit(p, ui, u); ++ui) {
                 const int d = ui & 1;
-                if (ui >= 2 && !warp_wait(&dempty[d], (uint32_t)((ui >> 1) - 1) & 1u, kStatusMmaWait, kNapDrain)) {
+                if (ui >= 2 && !warp_wait(&dempty[d], (uint32_t)((ui >> 1) - 1) & 1u, kStatusMmaWait, kNapDrain, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -650,11 +645,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 const uint32_t dcol = tmem + (uint32_t)((d * niss + w) * Mpad);
                 for (int t = u.t0; t < u.t1; ++t, ++g) {
                     const int a = aslot;
-                    if (!warp_wait(&afull[a], (uint32_t)awrap & 1u, kStatusTmaWait, kNapCritical)) {
+                    if (!warp_wait(&afull[a], (uint32_t)awrap & 1u, kStatusTmaWait, kNapCritical, p.wait_ns)) {
                         ok = false;
                         break;
                     }
-                    if (w == 0) RQ_TC_MARK(2, g);
                     tc_fence_after();
                     const uint32_t xs = base + (uint32_t)slot * p.stage_bytes;
                     const uint32_t acol = tmem + p.A0 + (uint32_t)a * ACOLS;
@@ -665,37 +659,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                                  (t != u.t0 || at != w) ? 1u : 0u);
                     mma_commit(&empty[slot]);
                     mma_commit(&aempty[a]);
-                    if (w == 0) RQ_TC_MARK(3, g);
                     if (++slot == R) slot = 0;
                     if (++aslot == AS) { aslot = 0; ++awrap; }
                 }
                 if (ok) mma_commit(&dfull[d]);
             }
             mma_commit(&mmadone[w]);
-            warp_wait(&mmadone[w], 0u, kStatusMmaWait, kNapDrain);      // no MMA in flight at teardown
+            warp_wait(&mmadone[w], 0u, kStatusMmaWait, kNapDrain, p.wait_ns);      // no MMA in flight at teardown
         }
     } else if (warp == 2) {
         // ------------------------------------------------------ tensor copies (one thread)
         if (lane == 0) {
             grid_dep_wait();                                 // x comes from earlier kernels
-            uint32_t g = 0;
-            int slot = 0, wrap = 0;
+            int slot = 0, wrap = 0, issued = 0;
             Unit u;
             bool ok = true;
             for (int ui = 0; ok && get_unit(p, ui, u); ++ui) {
                 const TcItem& it = p.it[u.item];
-                for (int t = u.t0; t < u.t1; ++t, ++g) {
-                    if (wrap && !nap_wait(&empty[slot], (uint32_t)(wrap - 1) & 1u, kStatusSlotWait, kNapLoader)) {
+                asm volatile("prefetch.tensormap [%0];" :: "l"(&it.cmap) : "memory");
+                asm volatile("prefetch.tensormap [%0];" :: "l"(&it.xmap) : "memory");
+                for (int t = u.t0; t < u.t1; ++t) {
+                    if (wrap && !nap_wait(&empty[slot], (uint32_t)(wrap - 1) & 1u, kStatusSlotWait, kNapLoader, p.wait_ns)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t st = base + (uint32_t)slot * p.stage_bytes;
-                    mbar_arrive_expect_tx(&full[slot], p.tx_bytes);
-                    tma_2d(st + p.codes_off, &it.cmap, t * RB, u.n0, &full[slot]);
-                    tma_3d(st, &it.xmap, 0, 0, t * NAT, &full[slot]);
-                    RQ_TC_MARK(0, g);
+                    if (!(p.test_flags & kTestNoCopies)) {
+                        const uint32_t st = base + (uint32_t)slot * p.stage_bytes;
+                        mbar_arrive_expect_tx(&full[slot], p.tx_bytes);
+                        tma_2d(st + p.codes_off, &it.cmap, t * RB, u.n0, &full[slot]);
+                        tma_3d(st, &it.xmap, 0, 0, t * NAT, &full[slot]);
+                        ++issued;
+                    }
                     if (++slot == R) { slot = 0; ++wrap; }
                 }
+            }
+            // Copies still in flight (consumers that gave up) land before the CTA leaves.
+            for (int s = 0; s < R && s < issued; ++s) {
+                const int uses = issued / R + (s < issued % R ? 1 : 0);
+                nap_wait(&full[s], (uint32_t)(uses - 1) & 1u, kStatusTmaWait, kNapDrain, p.wait_ns);
             }
         }
         __syncwarp();
@@ -704,7 +705,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         const int q = warp & 3, h = (warp - 3) >> 2;           // lane quarter, quarter of the stage's K
         const int r = 32 * q + lane;
         const uint32_t tl = (uint32_t)(32 * q) << 16;         // this warp's lane quarter
-        ScaleCursor<FMT, KS, MAXI> sc;
+        ScaleCursor<FMT, KS, TcArgs<MAXI>> sc;
         sc.start(&p, r, h);
         // scale FIFO: slot i is written and read at the same unrolled position,
         // so no register holding an in-flight load is ever copied
@@ -733,11 +734,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 if (!live) break;
                 const uint32_t s = sq[i] & sm[i];
                 sc.next(sq[i], sm[i]);
-                if (!warp_wait(&full[slot], (uint32_t)wrap & 1u, kStatusTmaWait, kNapCritical)) { ok = false; break; }
-                if (warp == 3 && lane == 0) RQ_TC_MARK(4, g);
+                if (!warp_wait(&full[slot], (uint32_t)wrap & 1u, kStatusTmaWait, kNapCritical, p.wait_ns)) { ok = false; break; }
                 const int a = aslot;
-                if (awrap && !warp_wait(&aempty[a], (uint32_t)(awrap - 1) & 1u, kStatusMmaWait, kNapCritical)) { ok = false; break; }
-                if (warp == 3 && lane == 0) RQ_TC_MARK(5, g);
+                if (awrap && !warp_wait(&aempty[a], (uint32_t)(awrap - 1) & 1u, kStatusMmaWait, kNapCritical, p.wait_ns)) { ok = false; break; }
                 const uint8_t* cs = smem + (size_t)slot * p.stage_bytes + p.codes_off;
                 const uint32_t ta = tmem + tl + p.A0 + (uint32_t)a * ACOLS + (uint32_t)h * QCOLS;
                 if (FMT == kFmtW4SB32) {                      // 64 weights: groups 2h, 2h+1 of the record
@@ -792,7 +791,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&afull[a]);
-                if (warp == 3 && lane == 0) RQ_TC_MARK(6, g);
                 if (++slot == R) { slot = 0; ++wrap; }
                 if (++aslot == AS) { aslot = 0; ++awrap; }
                 ++g;
@@ -812,8 +810,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         Unit u;
         for (int ui = 0; get_unit(p, ui, u); ++ui) {
             const int d = ui & 1;
-            if (!warp_wait(&dfull[d], (uint32_t)(ui >> 1) & 1u, kStatusMmaWait, kNapEpilogue)) break;
-            if (warp == 19 && lane == 0) RQ_TC_MARK(7, ui);
+            if (!warp_wait(&dfull[d], (uint32_t)(ui >> 1) & 1u, kStatusMmaWait, kNapEpilogue, p.wait_ns)) break;
             tc_fence_after();
             const TcItem& it = p.it[u.item];
             const int N = it.N, n = u.n0 + r;
@@ -1001,6 +998,8 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
     p.R = R;
     p.bar_off = (uint32_t)R * p.stage_bytes;
     const size_t smem = p.bar_off + bars + 1024;             // + alignment slack
+    p.wait_ns = wait_limit_ns();
+    p.test_flags = test_flags();
 
     auto kern = tc_kernel<FMT, KS, MAXI>;
     static unsigned long long attr_done = 0ull;

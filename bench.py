@@ -148,9 +148,8 @@ def oracle_sample(w, seconds: float, seed: int = 0):
         codes, scales = oracle.pack(m.fmt, g, a if m.n_cand > 1 else None, n_cand=m.n_cand,
                                     t_lo=0.7 if m.n_cand > 1 else 1.0)
         x = wl.bf16_bits(wl.activations(w, j, m.K, 1))
-        import weight_only_quantized_rq_b200 as rq_
-        cb, sb = rq_.rq_packed_size(m.fmt, m.K, m.N)
-        per_row = (cb + sb) / m.N
+        cshape, _, sshape = oracle.packed_shapes(m.fmt, m.K, m.N)
+        per_row = cshape[1] + (2 * sshape[1] if sshape else 0)          # packed bytes of one row
         shapes.append((m, codes, scales, x, rows, per_row))
     done_bytes, t0 = 0.0, time.perf_counter()
     reps = 0
@@ -165,6 +164,52 @@ def oracle_sample(w, seconds: float, seed: int = 0):
     desc = (f"oracle product (exact dequant + fp64 ascending-k sums) over 128 rows of each of the "
             f"{len(shapes)} matrix shapes of one layer, M=1, repeated {reps}x ({el:.1f} s)")
     return done_bytes / el / 1e9, desc, oracle.threads(), el
+
+
+def host_cpu():
+    """CPU model and the cores this process may run on."""
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return model, cores
+
+
+def oracle_pack_rate(w, seconds: float):
+    """The oracle's quantize-pack (the E[x^2]-weighted search of the method,
+    rwkv-quant article "Two presets and six sizes") over a few rows of each
+    matrix shape of one layer of the workload, repeated for about `seconds`:
+    weights per second."""
+    import numpy as np
+
+    import oracle
+    from weight_only_quantized_rq_b200 import workloads as wl
+    oracle.build()
+    sample = []
+    for j, layer, m in w.matrices():
+        if layer > 0:
+            break
+        rows = 8
+        sample.append((m, wl.random_matrix(20_000 + j, rows, m.K).numpy(), wl.act_sq(w, m.K)))
+    done, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        for m, W, a in sample:
+            oracle.pack(m.fmt, W, a if m.n_cand > 1 else None, n_cand=m.n_cand,
+                        t_lo=0.7 if m.n_cand > 1 else 1.0)
+            done += W.size
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return done / el, f"8 rows of each of the {len(sample)} matrix shapes of one layer, {reps}x ({el:.1f} s)"
 
 
 def run_reference(args, w, M):
@@ -310,8 +355,16 @@ def run_ours(args, w, M):
     # CPU baseline first, before heavy GPU work (rank 0, single GPU only)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
         v, desc, thr, _ = oracle_sample(w, args.cpu_seconds)
-        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": thr, "kind": "oracle", "sample": desc}
+        nthr = oracle.threads()
+        oracle.set_threads(1)
+        v1, desc1, _, _ = oracle_sample(w, args.cpu_seconds / 3)
+        oracle.set_threads(nthr)
+        model, aff = host_cpu()
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": thr, "kind": "oracle", "sample": desc,
+               "one_core": {"value": round(v1, 4), "unit": "GB/s", "sample": desc1},
+               "cpu_model": model, "cores_available": aff}
 
     mats = pack_workload(w, dev)
     prob = Problem(w, mats, M, dev)
@@ -449,6 +502,63 @@ def run_ours(args, w, M):
             variants[w2.name.split(" ")[0] + "/" + w2.per_layer[0].name] = measure(w2, mats2, list(w2.Ms))
             del mats2
             torch.cuda.empty_cache()
+    # quantize-pack (offline: the E[x^2]-weighted search, code emission and
+    # packing) of one layer of every configuration on the GPU, and the
+    # oracle's pack of a few rows of the same shapes on 1 core and on all
+    # cores (rank 0 only): weights per second
+    pack = None
+    if not args.quick:
+        pack = {}
+        for w2 in list(wl.WORKLOADS) + list(wl.VARIANTS):
+            shapes = [m for j2, layer2, m in w2.matrices() if layer2 == 0]
+            Ws = [wl.weights(w2, j2, m, device=str(dev)) for j2, layer2, m in w2.matrices() if layer2 == 0]
+            acts = [torch.from_numpy(wl.act_sq(w2, m.K)).to(dev) if m.n_cand > 1 else None for m in shapes]
+            outs = [rq.alloc_packed(m.fmt, m.K, m.N, dev) for m in shapes]
+
+            def pack_all(shapes=shapes, Ws=Ws, acts=acts, outs=outs):
+                for m, Wd, a, o in zip(shapes, Ws, acts, outs):
+                    rq.rq_quantize_pack(Wd, m.fmt, a, m.n_cand, 0.7 if m.n_cand > 1 else 1.0, 1.0, out=o,
+                                        stream=stream)
+            with torch.cuda.stream(stream):
+                pack_all()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                pack_all()
+                e1.record(stream)
+            e1.synchronize()
+            ms_p = e0.elapsed_time(e1)
+            nw = sum(m.K * m.N for m in shapes)
+            ent = {"matrices": [f"{m.fmt} {m.K}->{m.N} n_cand={m.n_cand}" for m in shapes],
+                   "gpu_ms": round(ms_p, 3), "gpu_Mweights_per_s": round(nw / (ms_p * 1e-3) / 1e6, 1)}
+            if rank == 0 and ws == 1 and not args.no_cpu_baseline:      # the CPU-baseline leg
+                import oracle
+                nthr = oracle.threads()
+                r_all, d_all = oracle_pack_rate(w2, 1.0)
+                oracle.set_threads(1)
+                r_one, d_one = oracle_pack_rate(w2, 1.0)
+                oracle.set_threads(nthr)
+                ent["oracle_Mweights_per_s"] = {"all_cores": round(r_all / 1e6, 3), "cores": nthr,
+                                                "one_core": round(r_one / 1e6, 3), "sample": d_all}
+                ent["gpu_over_oracle_all_cores"] = round(nw / (ms_p * 1e-3) / r_all, 1)
+            pack[w2.name.split(" ")[0]] = ent
+            del Ws, acts, outs
+        torch.cuda.empty_cache()
+    # config 1 as a single 768^2 product in one launch (launch-bound by
+    # construction; the configuration's line streams 2048 distinct copies)
+    single768 = None
+    if not args.quick:
+        w0 = wl.WORKLOADS[0]
+        m0 = w0.per_layer[0]
+        W0 = wl.weights(w0, 0, m0, device=str(dev))
+        p0 = rq.rq_quantize_pack(W0, m0.fmt, None, 1, 1.0, 1.0)
+        x0 = wl.activations(w0, 0, m0.K, 1, device=str(dev))
+        y0 = torch.empty(1, m0.N, device=dev)
+        f0 = capture(lambda: rq.rq_wgemm(x0, p0, y0, stream=stream))
+        ms0 = timed(f0, args.steps)
+        single768 = {"ms_per_call": round(ms0, 5), "calls_per_s": round(1e3 / ms0, 1),
+                     "GB_s": round(p0.nbytes / (ms0 * 1e-3) / 1e9, 2),
+                     "note": "one 313 KB matrix per launch: resident in L2 and bound by the launch, not by HBM"}
+        del W0, p0, x0, y0
     # the E[x^2] statistic of the scale search over a calibration batch of
     # 7.2B width (32768 rows x 4096 channels of bf16, 256 MB > L2)
     act_stats = None
@@ -543,6 +653,8 @@ def run_ours(args, w, M):
         "preset_variants": variants,
         "bf16_out": bf16_out,
         "act_stats": act_stats,
+        "pack": pack,
+        "single_768": single768,
         "gptq": gptq,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": prob.h2d,

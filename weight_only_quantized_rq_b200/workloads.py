@@ -59,8 +59,10 @@ class Workload:
 
 
 WORKLOADS = [
-    Workload(0, "w4g64-rtn-768 (RWKV-7 0.1B o_proj)",
-             (Matrix("o", 768, 768, "w4g64", 1),), 1, (1,), {768: "ch5x50"}),
+    # 2048 distinct copies (642 MB, more than four times the L2): one 313 KB
+    # matrix would sit in L2 and measure launch overhead, not the weight stream
+    Workload(0, "w4g64-rtn-768 (RWKV-7 0.1B o_proj) x2048 distinct",
+             (Matrix("o", 768, 768, "w4g64", 1),), 2048, (1,), {768: "ch5x50"}),
     Workload(1, "w8g16-aw-2048 (1.5B r/k/v/o x24, 0.1% outliers x10)",
              tuple(Matrix(n, 2048, 2048, "w8g16", 64, outliers=True) for n in "rkvo"),
              24, (1, 2, 4, 8), {}),

@@ -113,16 +113,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
-// Named barrier of n threads (id 1..15) that ANDs a flag over them: threads
-// that give up on a wait still take part, so every participant learns of it
-// and none is left waiting at the barrier.
-__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
-    uint32_t r;
-    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
-                 : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(n) : "memory");
-    return r != 0;
-}
-
 // ------------------------------------------------------ bulk async copy ---
 // One contiguous global -> shared copy completed on an mbarrier (the untiled
 // TMA form). dst, src and bytes must be multiples of 16. Loads with an L2

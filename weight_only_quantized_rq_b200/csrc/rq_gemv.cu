@@ -489,6 +489,7 @@ struct Ring {
     int s;                     // stage of the next group
     uint32_t ph;               // its phase parity
     unsigned long long lim;    // wait bound
+    volatile int* fail;        // raised by a warp whose wait gave up
 };
 
 // All groups of rows [ra, rb) of item `it` for this warp: waits for each
@@ -521,9 +522,11 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
                                                 mrows, lane, rbase, slice, red);
             if (KS > 1) {
                 // the k-slices of a team meet here; a slice whose wait gave up
-                // makes the whole team give up together (no warp is left at
-                // the barrier)
-                all = bar_and(1 + team, KS * 32, got);
+                // still arrives, after raising the CTA's give-up flag, and the
+                // whole team leaves together (no warp is left at the barrier)
+                if (!got) *ring.fail = 1;
+                asm volatile("bar.sync %0, %1;" :: "r"(1 + team), "r"(KS * 32) : "memory");
+                all = *ring.fail == 0;
                 if (all && slice == 0 && lane < RW * MT) {
                     const int r = lane / MT, m = lane - r * MT, rr = wfirst + r;
                     if (rr < rg && m < mrows) {
@@ -558,7 +561,9 @@ gemv_kernel(const Batch<MAXI> p) {
     const long long lo = (long long)blockIdx.x * p.total / gridDim.x;
     const long long hi = (long long)(blockIdx.x + 1) * p.total / gridDim.x;
 
+    __shared__ int s_fail;
     if (tid == 0) {
+        s_fail = 0;
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
@@ -662,6 +667,7 @@ gemv_kernel(const Batch<MAXI> p) {
     ring.s = 0;
     ring.ph = 0u;
     ring.lim = p.wait_ns;
+    ring.fail = &s_fail;
     int xi = 0;                                          // items done
     for (int i = i_first < 0 ? p.count : i_first; i < p.count; ++i) {
         const Item it = p.it[i];                         // this item's fields in registers
@@ -696,6 +702,7 @@ gemv_kernel(const Batch<MAXI> p) {
 constexpr int kSingleCtasPerSm = 1;
 constexpr int kBatchCtasPerSm = 2;
 constexpr size_t kSmemTarget = 72 * 1024;
+constexpr long long kWideBytes = 32ll << 20;          // single products from this size run as batches do
 constexpr size_t kSmemBatch = 112 * 1024;
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemAttr = kSmemLimit + 1024;
@@ -838,15 +845,19 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
             const size_t rd = it.KS > 1 ? round16((size_t)it.Rg * MT * it.KS * 4) : 0;
             red = rd > red ? rd : red;
         }
+        // A large single product (the 7.2B head: 302 MB) runs like a batch, two
+        // CTAs per SM with deeper rings; a small one keeps room for the next
+        // kernels of a dependent chain on the same SM.
+        const bool wide = count > 1 || total >= kWideBytes;
         SmemPlan sp;
-        if (!ok || !plan_smem(sb, xbb, red, count > 1 ? kSmemBatch : kSmemTarget, 6, sp)) {
+        if (!ok || !plan_smem(sb, xbb, red, wide ? kSmemBatch : kSmemTarget, 6, sp)) {
             if (MT == 2) continue;                       // retry one activation row per launch
             return cudaErrorInvalidValue;
         }
         p.total = total;
         p.wait_ns = wait_limit_ns();
         p.test_flags = test_flags();
-        int grid = sm_count() * (count > 1 ? kBatchCtasPerSm : kSingleCtasPerSm);
+        int grid = sm_count() * (wide ? kBatchCtasPerSm : kSingleCtasPerSm);
         if (count == 1 && grid > units_min) grid = (int)units_min;
         int stages = sp.stages;
         if (count == 1) {   // a single product needs no more stages than its largest CTA has groups

@@ -33,15 +33,17 @@ def _setup():
     assert rq.rq_device_status() == 0
 
 
-@pytest.mark.parametrize("fmt,M,kernel", [
-    ("w4g64", 1, "register GEMV"),
-    ("w4g64", 8, "tensor-core kernel"),
-    ("w8g16", 8, "tensor-core kernel"),
-    ("w5sb32", 1, "tensor-core kernel"),
-    ("w4g64", 64, "tensor-core kernel"),
+@pytest.mark.parametrize("fmt,M,K,kernel", [
+    ("w4g64", 1, 1024, "register GEMV"),
+    ("w4g64", 1, 8192, "register GEMV with rows split over k-slice warps"),
+    ("w8g16", 2, 4096, "register GEMV with rows split over k-slice warps"),
+    ("w4g64", 8, 1024, "tensor-core kernel"),
+    ("w8g16", 8, 1024, "tensor-core kernel"),
+    ("w5sb32", 1, 1024, "tensor-core kernel"),
+    ("w4g64", 64, 1024, "tensor-core kernel"),
 ])
-def test_waits_run_out_then_the_next_call_is_correct(fmt, M, kernel):
-    K, N = 1024, 700
+def test_waits_run_out_then_the_next_call_is_correct(fmt, M, K, kernel):
+    N = 700
     W = wl.random_matrix(3700, N, K).numpy()
     oc, osc = oracle.pack(fmt, W, None, n_cand=1, t_lo=1.0, t_hi=1.0)
     p = rq.alloc_packed(fmt, K, N)

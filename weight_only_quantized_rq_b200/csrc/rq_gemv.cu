@@ -489,7 +489,6 @@ struct Ring {
     int s;                     // stage of the next group
     uint32_t ph;               // its phase parity
     unsigned long long lim;    // wait bound
-    volatile int* fail;        // raised by a warp whose wait gave up
 };
 
 // All groups of rows [ra, rb) of item `it` for this warp: waits for each
@@ -499,7 +498,7 @@ struct Ring {
 // setup stays outside the group loop. False if a bounded wait gave up.
 template <int FMT, int MT, int RW, int TT, int YB>
 __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& ring, uint32_t x_s, int m0,
-                                          int mrows, int warp, int lane) {
+                                          int mrows, int warp, int lane, int& g_fail) {
     const int T = TT ? TT : it.T, KS = it.KS, Rg = it.Rg;
     const int slice = warp % KS;                         // k-slice of this warp (KS > 1 only when T == 32)
     const int team = warp / KS;                          // warps team*KS .. team*KS+KS-1 share rows
@@ -508,7 +507,7 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
     const int wfirst = wteam * RW;                       // first row of this warp in a group
     for (int g0 = ra; g0 < rb; g0 += Rg) {
         const int s = ring.s;
-        const bool got = mbar_wait_bounded(&ring.full[s], ring.ph, kStatusTmaWait, 0u, ring.lim);
+        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&ring.full[s], ring.ph, kStatusTmaWait, 0u, ring.lim));
         if (++ring.s == ring.stages) {                   // next stage and its phase parity
             ring.s = 0;
             ring.ph ^= 1u;
@@ -524,9 +523,7 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
                 // the k-slices of a team meet here; a slice whose wait gave up
                 // still arrives, after raising the CTA's give-up flag, and the
                 // whole team leaves together (no warp is left at the barrier)
-                if (!got) *ring.fail = 1;
                 asm volatile("bar.sync %0, %1;" :: "r"(1 + team), "r"(KS * 32) : "memory");
-                all = *ring.fail == 0;
                 if (all && slice == 0 && lane < RW * MT) {
                     const int r = lane / MT, m = lane - r * MT, rr = wfirst + r;
                     if (rr < rg && m < mrows) {
@@ -538,11 +535,37 @@ __device__ __forceinline__ bool gemv_item(const Item& it, int ra, int rb, Ring& 
                 }
             }
         }
-        if (!all) return false;
+        if (!all) {
+            g_fail = g0;                                 // this group's barrier was met; the rest are not
+            return false;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);     // stage consumed
     }
     return true;
+}
+
+// After a bounded wait gave up in the group at row g_fail of item i0, a
+// consumer warp still owes its team its part in every later k-slice barrier
+// that its teammates, which may still be computing, will reach: it takes
+// each of them in turn (a barrier instance must complete before the warp
+// counts toward the next), then leaves. Never taken unless a wait ran out.
+template <int MAXI>
+__device__ __noinline__ void gemv_give_up(const Batch<MAXI>& p, int i0, int g_fail, long long lo, long long hi,
+                                          int warp) {
+    for (int i = i0; i < p.count; ++i) {
+        const Item& it = p.it[i];
+        if (it.cost0 >= hi) break;
+        if (it.cost1 <= lo) continue;
+        int ua, ub;
+        item_units(it, lo, hi, ua, ub);
+        const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
+        if (ra >= rb || it.KS <= 1) continue;
+        const int team = warp / it.KS, wfirst = team * (32 / it.T) * it.RW;
+        for (int g0 = (i == i0 ? g_fail + it.Rg : ra); g0 < rb; g0 += it.Rg)
+            if (wfirst < min(it.Rg, rb - g0))
+                asm volatile("bar.sync %0, %1;" :: "r"(1 + team), "r"(it.KS * 32) : "memory");
+    }
 }
 
 // Resident CTAs per SM the register budget is sized for.
@@ -551,7 +574,7 @@ constexpr int min_blocks(int) { return kConsumerWarps <= 12 ? 2 : 1; }
 // YB: outputs rounded once to bf16 (1) or fp32 (0), fixed per launch.
 template <int FMT, int MT, int MAXI, int YB>
 __global__ void __launch_bounds__(kThreads, min_blocks(MT))
-gemv_kernel(const Batch<MAXI> p) {
+gemv_kernel(const __grid_constant__ Batch<MAXI> p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
@@ -561,9 +584,7 @@ gemv_kernel(const Batch<MAXI> p) {
     const long long lo = (long long)blockIdx.x * p.total / gridDim.x;
     const long long hi = (long long)(blockIdx.x + 1) * p.total / gridDim.x;
 
-    __shared__ int s_fail;
     if (tid == 0) {
-        s_fail = 0;
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
@@ -667,7 +688,6 @@ gemv_kernel(const Batch<MAXI> p) {
     ring.s = 0;
     ring.ph = 0u;
     ring.lim = p.wait_ns;
-    ring.fail = &s_fail;
     int xi = 0;                                          // items done
     for (int i = i_first < 0 ? p.count : i_first; i < p.count; ++i) {
         const Item it = p.it[i];                         // this item's fields in registers
@@ -678,19 +698,26 @@ gemv_kernel(const Batch<MAXI> p) {
         const int ra = ua * it.rho, rb = min(ub * it.rho, it.N);
         if (ra >= rb) continue;
         const int b = xi % p.nxb;
-        if (!mbar_wait_bounded(&xfull[b], (xi / p.nxb) & 1, kStatusXWait, 0u, p.wait_ns)) return;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&xfull[b], (xi / p.nxb) & 1, kStatusXWait, 0u, p.wait_ns))) {
+            gemv_give_up(p, i, ra - it.Rg, lo, hi, warp);  // owes every barrier of this item and the later ones
+            return;
+        }
         const uint32_t x_s = smem_s + p.x_off + (uint32_t)b * p.x_bytes;
         bool ok;
+        int g_fail = 0;
         if (it.T == 32) {                                // whole-warp teams: the common case
-            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                              : gemv_item<FMT, MT, 1, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
+            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
+                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
+                              : gemv_item<FMT, MT, 1, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail);
         } else {
-            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane)
-                              : gemv_item<FMT, MT, 1, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane);
+            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
+                 : it.RW == 2 ? gemv_item<FMT, MT, 2, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
+                              : gemv_item<FMT, MT, 1, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail);
         }
-        if (!ok) return;
+        if (!ok) {
+            gemv_give_up(p, i, g_fail, lo, hi, warp);
+            return;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&xempty[b]);          // staged x released
         ++xi;

@@ -80,7 +80,7 @@ constexpr int kMaxAS = 8;           // A slots at most (the accumulators take th
 constexpr int kDqThreads = 512;     // warps 3-18
 constexpr int kEpiThreads = 128;    // warps 19-22
 constexpr int kTcThreads = 736;
-constexpr int kScaleAhead = 4;      // stages of scales held in registers ahead of use
+constexpr int kScaleAhead = 2;      // stages of scales held in registers ahead of use
 constexpr size_t kTcSmemMax = 227 * 1024;
 
 struct __align__(64) TcItem {       // one product of a launch

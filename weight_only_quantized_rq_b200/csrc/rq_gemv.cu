@@ -383,50 +383,67 @@ __device__ __forceinline__ void gemv_group(const Item& it, uint32_t st_s, int g0
     } else {
         // int8: 32 code bytes per row and half-chunk h = groups 2h, 2h+1 of
         // 16 (two scales) or half of group h/2 of 64 (one scale); x as fp32
-        // quads, 8 per half-chunk
+        // quads, 8 per half-chunk. Rows are taken two at a time, so each x
+        // quad loaded from shared memory serves two rows (halving the x
+        // traffic, which is what limits two activation rows) within the
+        // register budget.
+        constexpr int RB = MT == 1 || RW < 2 ? 1 : 2;
+        constexpr int UW = MT == 1 ? U : 1;              // two half-chunks per iteration spill at MT = 2
         uint32_t ca[RW], sa[RW];
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
             ca[r] = st_s + (uint32_t)(rbase + r) * crb + (uint32_t)li * 32u;
             sa[r] = ssc_s + (uint32_t)(rbase + r) * srb;
         }
-        for (int hj = 0; hj < HJ; hj += U) {
+        for (int hj = 0; hj < HJ; hj += UW) {
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                if (u > 0 && hj + u >= HJ) break;
-                const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
+          for (int u = 0; u < UW; ++u) {
+            if (u > 0 && hj + u >= HJ) break;
+            const uint32_t dh = (uint32_t)(hoff + hj + u) * (uint32_t)T;
+            const uint32_t hc = dh + (uint32_t)li;           // this lane's half-chunk of the row
 #pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    const uint4 c0 = lds128_a(ca[r] + dh * 32u);
-                    const uint4 c1 = lds128_a(ca[r] + dh * 32u + 16u);
-                    const uint32_t hc = dh + (uint32_t)li;   // this lane's half-chunk of the row
-                    const uint32_t sp = FMT == kFmtW8G64 ? lds16_a(sa[r] + ((hc >> 1) << 1)) * 0x10001u
-                                                         : lds32_a(sa[r] + hc * 4u);
-                    const float s0 = __half2float(__ushort_as_half((unsigned short)(sp & 0xffffu)));
-                    const float s1 = __half2float(__ushort_as_half((unsigned short)(sp >> 16)));
+            for (int r0 = 0; r0 < RW; r0 += RB) {
+                uint32_t sp[RB];
 #pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        float a[MT];
+                for (int r = 0; r < RB; ++r)
+                    sp[r] = FMT == kFmtW8G64 ? lds16_a(sa[r0 + r] + ((hc >> 1) << 1)) * 0x10001u
+                                             : lds32_a(sa[r0 + r] + hc * 4u);
 #pragma unroll
-                        for (int m = 0; m < MT; ++m) a[m] = 0.0f;
+                for (int g = 0; g < 2; ++g) {                // 16-weight halves of the half-chunk
+                    uint4 c[RB];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            float f[4];
-                            unpack_w8(word_of(g ? c1 : c0, i), f);
+                    for (int r = 0; r < RB; ++r) c[r] = lds128_a(ca[r0 + r] + dh * 32u + 16u * (uint32_t)g);
+                    float a[RB][MT];
 #pragma unroll
-                            for (int m = 0; m < MT; ++m) {
-                                const float4 xv = lds128f_a(xa0 + dh * 16u + (uint32_t)(m * 8 + g * 4 + i) * xstride);
-                                a[m] = fmaf(f[0], xv.x, a[m]);
-                                a[m] = fmaf(f[1], xv.y, a[m]);
-                                a[m] = fmaf(f[2], xv.z, a[m]);
-                                a[m] = fmaf(f[3], xv.w, a[m]);
+                    for (int r = 0; r < RB; ++r)
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) a[r][m] = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float f[RB][4];
+#pragma unroll
+                        for (int r = 0; r < RB; ++r) unpack_w8(word_of(c[r], i), f[r]);
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) {
+                            const float4 xv = lds128f_a(xa0 + dh * 16u + (uint32_t)(m * 8 + g * 4 + i) * xstride);
+#pragma unroll
+                            for (int r = 0; r < RB; ++r) {
+                                a[r][m] = fmaf(f[r][0], xv.x, a[r][m]);
+                                a[r][m] = fmaf(f[r][1], xv.y, a[r][m]);
+                                a[r][m] = fmaf(f[r][2], xv.z, a[r][m]);
+                                a[r][m] = fmaf(f[r][3], xv.w, a[r][m]);
                             }
                         }
+                    }
 #pragma unroll
-                        for (int m = 0; m < MT; ++m) yacc[r][m] = fmaf(g ? s1 : s0, a[m], yacc[r][m]);
+                    for (int r = 0; r < RB; ++r) {
+                        const float sg = __half2float(__ushort_as_half((unsigned short)(g ? sp[r] >> 16 : sp[r] & 0xffffu)));
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) yacc[r0 + r][m] = fmaf(sg, a[r][m], yacc[r0 + r][m]);
                     }
                 }
             }
+          }
         }
     }
     if (T == 32 && RW == 4) {
@@ -705,12 +722,15 @@ gemv_kernel(const __grid_constant__ Batch<MAXI> p) {
         const uint32_t x_s = smem_s + p.x_off + (uint32_t)b * p.x_bytes;
         bool ok;
         int g_fail = 0;
+        // int8 at two activation rows keeps at most two rows per lane team (four
+        // would not fit the register budget); that case is never planned
+        constexpr int RW4 = is_w8(FMT) && MT == 2 ? 2 : 4;
         if (it.T == 32) {                                // whole-warp teams: the common case
-            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
+            ok = it.RW == 4   ? gemv_item<FMT, MT, RW4, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
                  : it.RW == 2 ? gemv_item<FMT, MT, 2, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
                               : gemv_item<FMT, MT, 1, 32, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail);
         } else {
-            ok = it.RW == 4   ? gemv_item<FMT, MT, 4, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
+            ok = it.RW == 4   ? gemv_item<FMT, MT, RW4, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
                  : it.RW == 2 ? gemv_item<FMT, MT, 2, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail)
                               : gemv_item<FMT, MT, 1, 0, YB>(it, ra, rb, ring, x_s, p.m0, p.mrows, warp, lane, g_fail);
         }
@@ -853,7 +873,9 @@ cudaError_t launch_batch(const WgemmArgs* a, int count, cudaStream_t st) {
         for (int i = 0; i < count && ok; ++i) {
             Item& it = p.it[i];
             size_t s1;
-            if (!plan_item(FMT, a[i].K, a[i].N, MT, rw_allowed(FMT, a[i].K), it, s1)) {
+            int rw = rw_allowed(FMT, a[i].K);
+            if (is_w8(FMT) && MT == 2 && rw > 2) rw = 2;   // the register budget (see the kernel's dispatch)
+            if (!plan_item(FMT, a[i].K, a[i].N, MT, rw, it, s1)) {
                 ok = false;
                 break;
             }

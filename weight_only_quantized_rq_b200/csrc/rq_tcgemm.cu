@@ -41,9 +41,18 @@
 //    two accumulators that the epilogue adds in a fixed order. Warp 0 also
 //    allocates tensor memory. Warp 2 issues the tensor copies; warps 3-18
 //    dequantize (warp w owns tensor-memory lanes 32 (w % 4) .. +31, i.e. one
-//    weight row per thread, and a quarter of each stage's K: four warps per
-//    SM sub-partition hide each other's latency); warps 19-22 read D back with
-//    tcgen05.ld and store y.
+//    weight row per thread); warps 19-22 read D back with tcgen05.ld and
+//    store y.
+//  * Dequantizing groups: where the A ring has room (3 or more slots; 5 or
+//    more at 128-K stages), the sixteen dequantizing warps form 2 (or 4)
+//    groups that take the stages in turn, each warp writing 2 (or 4) K
+//    quarters of its group's stage. When all sixteen warps shared every
+//    stage, they met every barrier together and the SM sub-partitions sat
+//    idle between stages (traced: about 1.8 thousand cycles per 256-K stage,
+//    half of them outside the arithmetic); with groups out of phase one
+//    group's waits overlap another's arithmetic, and a warp meets fewer
+//    barriers per weight. Where the ring is smaller (M > 32 at 256-K stages,
+//    M > 64 at 128-K stages) all sixteen share each stage, a quarter each.
 //  * int4: a lop3 with mask and exponent pattern places nibble pairs in fp16
 //    mantissas: (1024 + u) for the low nibble of a byte, (64 + u) for the high
 //    nibble; fma.rn.f32.f16 against the fp16 scale and an exact fp32 offset
@@ -83,6 +92,7 @@ constexpr int kTcThreads = 736;
 constexpr int kScaleAhead = 2;      // stages of scales held in registers ahead of use
 constexpr size_t kTcSmemMax = 227 * 1024;
 
+
 struct __align__(64) TcItem {       // one product of a launch
     CUtensorMap cmap;               // codes plane: uint8 [N][crb], box [128 rows][RB bytes], swizzled
     CUtensorMap xmap;               // x: bf16 [M][K] viewed as [K/64][M][64], box [KS/64][xrows][64]
@@ -105,6 +115,7 @@ struct TcArgs {
     int niss;                       // MMA-issuing warps (two accumulators when Mpad <= 64)
     int AS;                         // A slots in tensor memory
     uint32_t A0;                    // first tensor-memory column of the A slots (after 2 * niss accumulators)
+    int ng;                         // groups of dequantizing warps that take the stages in turn (1, 2 or 4)
     uint32_t stage_bytes, x_atom, codes_off, bar_off, tx_bytes;
     unsigned long long wait_ns;     // bound of every device wait
     int test_flags;                 // kTestNoCopies: the copy thread issues nothing (tests the waits)
@@ -231,6 +242,11 @@ __device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
 __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
     uint32_t v;
     asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ldg_nc_u64(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
     return v;
 }
 // fp32 pair -> bf16x2 (round to nearest even), lo in the low half.
@@ -571,6 +587,165 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsign
 // Sleep between phase tests, by waiter (ns; 0 = suspending try_wait).
 constexpr unsigned kNapCritical = 0, kNapLoader = 64, kNapEpilogue = 512, kNapDrain = 256;
 
+// Dequantizing warps in NG groups (2 or 4) that take the CTA's stages in
+// turn: in its group's stage, warp (q, h) writes rows 32q .. 32q+31 of the
+// NG consecutive K quarters from (h mod 4/NG) NG on (64 weights per quarter
+// at 256-K int4 stages, 32 otherwise). Compared with all sixteen warps
+// sharing every stage, a warp meets 1/NG as many barriers per weight, and
+// the groups run out of phase, so one group's waits overlap another's
+// arithmetic. Needs more than NG A slots. A wait that runs out ends the role
+// (its status bit is set).
+template <int FMT, int KS, int NG, int MAXI>
+__device__ __forceinline__ void dequant_groups(const TcArgs<MAXI>& p, const uint8_t* smem, uint32_t tmem,
+                                               uint64_t* full, uint64_t* afull, uint64_t* aempty, int warp,
+                                               int lane) {
+    constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : is_w8(FMT) ? KS : FMT == kFmtW6G16 ? KS / 64 * 48
+                                                                   : sb_record(FMT);   // code bytes per row and stage
+    constexpr uint32_t QCOLS = KS / 8;                       // tensor-memory columns per K quarter
+    constexpr int SUBS = 4 / NG;                             // warps of a group per lane quarter
+    const int q = warp & 3, hh = (warp - 3) >> 2, grp = hh / SUBS, h0 = (hh % SUBS) * NG;
+    const int r = 32 * q + lane;
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    const int R = p.R, AS = p.AS;
+    Unit u;
+    int ui = 0, t = 0, slot = 0, wrap = 0, aslot = 0, awrap = 0;
+    bool live = get_unit(p, 0, u);
+    if (live) t = u.t0;
+    auto step = [&]() {                                      // to the CTA's next stage
+        if (++slot == R) { slot = 0; ++wrap; }
+        if (++aslot == AS) { aslot = 0; ++awrap; }
+        if (++t >= u.t1) {
+            live = get_unit(p, ++ui, u);
+            if (live) t = u.t0;
+        }
+    };
+    // Scale words of this thread's row for quarters h0 .. h0 + NG - 1 at the
+    // current stage, loaded together: group-16 formats two fp16 scales per
+    // quarter (8 bytes per pair of quarters); int4 g64 at 256-K stages one per
+    // quarter (NG = 2: one 4-byte load); g64 at 128-K stages one per two
+    // quarters. The superblock formats carry theirs in the records. Rows past
+    // N and groups past K get zero (and nothing is read there).
+    constexpr int NW = is_sb(FMT) ? 1 : sym_group(FMT) == 16 ? NG : 1;
+    auto load_scales = [&](uint32_t (&w)[NW]) {
+#pragma unroll
+        for (int k = 0; k < NW; ++k) w[k] = 0u;
+        if constexpr (!is_sb(FMT)) {
+            const TcItem& it = p.it[u.item];
+            const int n = u.n0 + r;
+            if (n >= it.N) return;
+            const int groups = it.K / sym_group(FMT);
+            const uint8_t* row = it.scales + (size_t)n * it.srb;
+            if constexpr (sym_group(FMT) == 16) {            // K % 64 == 0: pairs of quarters are whole or absent
+#pragma unroll
+                for (int k = 0; k < NG; k += 2) {
+                    const int gi = 8 * t + 2 * (h0 + k);
+                    if (gi < groups) {
+                        const uint2 v = ldg_nc_u64(row + 2 * gi);
+                        w[k] = v.x;
+                        w[k + 1] = v.y;
+                    }
+                }
+            } else if constexpr (KS == 256) {                // K % 256 == 0: both groups exist
+                w[0] = ldg_nc_u32(row + 2 * (4 * t + h0));
+            } else {
+                const int gi = 2 * t + (h0 >> 1);
+                if (NG == 4 && gi + 1 < groups && (it.srb & 3u) == 0u) w[0] = ldg_nc_u32(row + 2 * gi);
+                else if (gi < groups)
+                    w[0] = ldg_nc_u16(row + 2 * gi) | (NG == 4 && gi + 1 < groups ? ldg_nc_u16(row + 2 * gi + 2) << 16 : 0u);
+            }
+        }
+    };
+    auto scale_at = [](const uint32_t (&w)[NW], int j) -> uint32_t {
+        if constexpr (is_sb(FMT)) return 0u;
+        else if constexpr (sym_group(FMT) == 16) return w[j];
+        else if constexpr (KS == 256) return j & 1 ? w[0] >> 16 : w[0] & 0xffffu;
+        else return NG == 4 && j >= 2 ? w[0] >> 16 : w[0] & 0xffffu;
+    };
+    for (int k = 0; k < grp && live; ++k) step();
+    uint32_t sw[NW];
+    if (live) load_scales(sw);
+    while (live) {
+        if (!warp_wait(&full[slot], (uint32_t)wrap & 1u, kStatusTmaWait, kNapCritical, p.wait_ns)) return;
+        const int a = aslot;
+        if (awrap && !warp_wait(&aempty[a], (uint32_t)(awrap - 1) & 1u, kStatusMmaWait, kNapCritical, p.wait_ns))
+            return;
+        const uint8_t* cs = smem + (size_t)slot * p.stage_bytes + p.codes_off;
+        const uint32_t ta0 = tmem + tl + p.A0 + (uint32_t)a * (KS / 2);
+        // the stage's code loads first, so that their latency overlaps the
+        // bookkeeping below (a tensor-memory store would order later
+        // shared-memory loads after it)
+        uint4 hd = make_uint4(0u, 0u, 0u, 0u), c[NG][2];
+        uint32_t pl[NG][4];
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+            const int hq = h0 + j;
+            if constexpr (is_sb(FMT)) {                      // 64 weights: groups 2hq, 2hq+1 of the record
+                if (j == 0) hd = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, 0));
+                c[j][0] = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, 1 + 2 * hq));
+                c[j][1] = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, 2 + 2 * hq));
+                const uint32_t pp = code_pos<RB>(r, 0) + 144u + (FMT == kFmtW6SB32 ? 16u : 8u) * (uint32_t)hq;
+                if constexpr (FMT == kFmtW6SB32) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(cs + pp);
+                    pl[j][0] = v.x; pl[j][1] = v.y; pl[j][2] = v.z; pl[j][3] = v.w;
+                } else if constexpr (FMT == kFmtW5SB32) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(cs + pp);
+                    pl[j][0] = v.x; pl[j][1] = v.y; pl[j][2] = 0u; pl[j][3] = 0u;
+                }
+            } else if constexpr (FMT == kFmtW4G64 && KS == 128) {   // 32 weights: chunk hq, half a group
+                c[j][0] = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, hq));
+            } else if constexpr (FMT == kFmtW6G16) {          // 32 weights: two groups of 16
+                c[j][0] = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, 3 * (hq >> 1) + (hq & 1)));
+                const uint2 v = *reinterpret_cast<const uint2*>(cs + code_pos<RB>(r, 3 * (hq >> 1) + 2) +
+                                                                8u * (uint32_t)(hq & 1));
+                pl[j][0] = v.x; pl[j][1] = v.y;
+            } else {                                          // int4 at 256-K stages (64 weights) or int8 (32):
+                c[j][0] = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, 2 * hq));   // chunks 2hq, 2hq+1
+                c[j][1] = *reinterpret_cast<const uint4*>(cs + code_pos<RB>(r, 2 * hq + 1));
+            }
+        }
+        uint32_t sc[NG];
+#pragma unroll
+        for (int j = 0; j < NG; ++j) sc[j] = scale_at(sw, j);
+#pragma unroll
+        for (int k = 0; k < NG; ++k)                         // to this group's next stage
+            if (live) step();
+        if (live) load_scales(sw);                           // loads while this stage is dequantized
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+            const int hq = h0 + j;
+            const uint32_t ta = ta0 + (uint32_t)hq * QCOLS;
+            if constexpr (is_sb(FMT)) {
+                uint32_t o[32];
+                if constexpr (FMT == kFmtW4SB32) dq_sb32(hd, c[j][0], c[j][1], hq, o);
+                else dq_sbw<FMT == kFmtW6SB32 ? 6 : 5>(hd, c[j][0], c[j][1], pl[j], hq, o);
+                tmem_st32(ta, o);
+            } else if constexpr (FMT == kFmtW4G64 && KS == 256) {
+                const uint32_t wv[8] = {c[j][0].x, c[j][0].y, c[j][0].z, c[j][0].w,
+                                        c[j][1].x, c[j][1].y, c[j][1].z, c[j][1].w};
+                uint32_t o[32];
+                dq_w4<8>(wv, (uint16_t)sc[j], o);
+                tmem_st32(ta, o);
+            } else if constexpr (FMT == kFmtW4G64) {
+                const uint32_t wv[4] = {c[j][0].x, c[j][0].y, c[j][0].z, c[j][0].w};
+                uint32_t o[16];
+                dq_w4<4>(wv, (uint16_t)sc[j], o);
+                tmem_st16(ta, o);
+            } else if constexpr (FMT == kFmtW6G16) {
+                uint32_t o[16];
+                dq_w6(c[j][0], make_uint2(pl[j][0], pl[j][1]), sc[j], o);
+                tmem_st16(ta, o);
+            } else {
+                uint32_t o[16];
+                dq_w8(c[j], FMT == kFmtW8G64 ? sc[j] * 0x10001u : sc[j], o);   // g64: one scale for both halves
+                tmem_st16(ta, o);
+            }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&afull[a]);
+    }
+}
+
 template <int FMT, int KS, int MAXI>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcArgs<MAXI> p) {
     constexpr int RB = FMT == kFmtW4G64 ? KS / 2 : is_w8(FMT) ? KS : FMT == kFmtW6G16 ? KS / 64 * 48
@@ -601,7 +776,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             mbar_init(&empty[s], (uint32_t)niss);
         }
         for (int a = 0; a < AS; ++a) {
-            mbar_init(&afull[a], kDqThreads);
+            mbar_init(&afull[a], (uint32_t)(kDqThreads / p.ng));
             mbar_init(&aempty[a], (uint32_t)niss);
         }
         for (int d = 0; d < 2; ++d) {
@@ -700,6 +875,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             }
         }
         __syncwarp();
+    } else if (KS == 128 && warp <= 18 && p.ng == 4) {             // 256-K stages have at most 3 A slots
+        dequant_groups<FMT, KS, KS == 128 ? 4 : 2>(p, smem, tmem, full, afull, aempty, warp, lane);
+    } else if (warp <= 18 && p.ng == 2) {
+        dequant_groups<FMT, KS, 2>(p, smem, tmem, full, afull, aempty, warp, lane);
     } else if (warp <= 18) {
         // ------------------------------------------------------ dequantize into tensor memory
         const int q = warp & 3, h = (warp - 3) >> 2;           // lane quarter, quarter of the stage's K
@@ -972,6 +1151,9 @@ cudaError_t launch_fmt_tc(const WgemmArgs* a, int count, cudaStream_t st) {
     p.AS = (int)((kTmemCols - p.A0) / (KS / 2));
     if (p.AS > kMaxAS) p.AS = kMaxAS;
     if (p.AS < 2) return cudaErrorInvalidValue;
+    // dequantizing groups: as many as the A slots allow (each group holds one
+    // slot while it works, the MMA at least one more)
+    p.ng = KS == 128 && p.AS >= 5 ? 4 : p.AS >= 3 ? 2 : 1;
     const int sms = sm_count();
     p.split = 1;
     if (count == 1 && units < sms / 2) {                     // too few tiles: split K over a cluster
@@ -1037,7 +1219,7 @@ cudaError_t launch_chunk(const WgemmArgs* a, int count, cudaStream_t st) {
     if constexpr (is_sb(FMT)) {                             // K % 256 == 0: one record per row and stage
         return count == 1 ? launch_fmt_tc<FMT, 256, 1>(a, 1, st) : launch_fmt_tc<FMT, 256, kTcMaxItems>(a, count, st);
     } else {
-        if (FMT == kFmtW4G64) {
+        if constexpr (FMT == kFmtW4G64) {
             bool wide = a[0].M <= 64;
             for (int i = 0; i < count; ++i) wide = wide && (a[i].K % 256 == 0);
             if (wide)

@@ -144,6 +144,64 @@ __device__ __forceinline__ int first_item(const Batch<MAXI>& p, long long lo, lo
 // consumers and the stager after staging a CTA's first item).
 constexpr int kCoopBarrier = 15;
 
+// g64 unit sums: the even-k and odd-k fp32 sums of a 64-value unit are formed
+// in one fixed order whichever threads stage it -- each 8-value chunk summed
+// in k order, then the chunk sums as the tree ((c0 + c1) + (c2 + c3)) +
+// ((c4 + c5) + (c6 + c7)) -- so the staged records, and the products, do
+// not depend on how a launch splits the staging.
+__device__ __forceinline__ float tree8(const float (&c)[8]) {
+    return __fadd_rn(__fadd_rn(__fadd_rn(c[0], c[1]), __fadd_rn(c[2], c[3])),
+                     __fadd_rn(__fadd_rn(c[4], c[5]), __fadd_rn(c[6], c[7])));
+}
+
+// g64 staging with eight threads per unit (one 16-byte chunk each): for a
+// CTA's first item, staged by all nthreads (a multiple of 32) threads right
+// after the dependency wait, where the latency of the x loads and of one
+// thread's pass over 64 values is on the critical path of a dependent launch.
+// Rounds are uniform over the threads, so every shuffle has all lanes.
+template <int MT>
+__device__ __forceinline__ void stage_x_g64_wide(const Item& it, int m0, int mrows, uint8_t* xb, int t, int nthreads) {
+    const int G = it.K >> 6, nu = MT * G;
+    uint8_t* meta = xb + xvals_bytes(kFmtW4G64, it.K, MT);
+    const int grp = t >> 3, sub = t & 7, ngrp = nthreads >> 3;
+    for (int base = 0; base < nu; base += ngrp) {
+        const int i = base + grp;
+        const bool act = i < nu;
+        const int m = act ? i / G : 0, g = act ? i - m * G : 0;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (act && m < mrows)
+            v = __ldg(reinterpret_cast<const uint4*>(it.x + (size_t)(m0 + m) * it.K + (size_t)g * 64) + sub);
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t mb = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+        const int e = mb != 0u ? min(126, max(-126, 14 - ((int)(mb >> 7) - 127))) : 0;
+        const float up = __int_as_float((e + 127) << 23), f = __int_as_float((127 - e) << 23);
+        float se = 0.0f, so = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
+            const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+            se = __fadd_rn(se, __half2float(a));
+            so = __fadd_rn(so, __half2float(b));
+            w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {                // the tree of tree8, one level per step
+            se = __fadd_rn(se, __shfl_xor_sync(0xffffffffu, se, o));
+            so = __fadd_rn(so, __shfl_xor_sync(0xffffffffu, so, o));
+        }
+        if (act) {
+            reinterpret_cast<uint4*>(xb)[((size_t)m * 8 + sub) * G + g] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (sub == 0)
+                reinterpret_cast<float2*>(meta)[(size_t)m * G + g] =
+                    make_float2(__fmaf_rn(1032.0f, se, __fmul_rn(72.0f, so)), f);
+        }
+    }
+}
+
 template <int FMT, int MT>
 __device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8_t* xb, int first, int stride) {
     constexpr bool kW4 = !is_w8(FMT);
@@ -170,15 +228,22 @@ __device__ __forceinline__ void stage_x(const Item& it, int m0, int mrows, uint8
             for (int j = 0; j < 32; ++j) mb = max(mb, max(w[j] & 0x7fffu, (w[j] >> 16) & 0x7fffu));
             const int e = mb != 0u ? min(126, max(-126, 14 - ((int)(mb >> 7) - 127))) : 0;
             const float up = __int_as_float((e + 127) << 23), f = __int_as_float((127 - e) << 23);
-            float se = 0.0f, so = 0.0f;
+            float ce[8], co[8];                          // per 8-value chunk, in k order
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
-                const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
-                se = __fadd_rn(se, __half2float(a));
-                so = __fadd_rn(so, __half2float(b));
-                w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+            for (int q = 0; q < 8; ++q) {
+                ce[q] = 0.0f;
+                co[q] = 0.0f;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = 4 * q + jj;
+                    const __half a = __float2half_rn(__fmul_rn(bf16lo_f32(w[j]), up));
+                    const __half b = __float2half_rn(__fmul_rn(bf16hi_f32(w[j]), up));
+                    ce[q] = __fadd_rn(ce[q], __half2float(a));
+                    co[q] = __fadd_rn(co[q], __half2float(b));
+                    w[j] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+                }
             }
+            const float se = tree8(ce), so = tree8(co);
             uint4* dst = reinterpret_cast<uint4*>(xb) + (size_t)m * 8 * G + g;
 #pragma unroll
             for (int q = 0; q < 8; ++q) dst[(size_t)q * G] = v[q];
@@ -665,7 +730,10 @@ gemv_kernel(const __grid_constant__ Batch<MAXI> p) {
     if (warp == kStagerWarp) {                           // x of each item into alternating buffers
         grid_dep_wait();                                 // x is written by the previous kernel
         if (i_first < 0) return;
-        stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, kConsumerWarps * 32 + lane, kCoop);
+        if constexpr (FMT == kFmtW4G64)
+            stage_x_g64_wide<MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, kConsumerWarps * 32 + lane, kCoop);
+        else
+            stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, kConsumerWarps * 32 + lane, kCoop);
         asm volatile("bar.sync %0, %1;" :: "n"(kCoopBarrier), "n"(kCoop) : "memory");
         mbar_arrive(&xfull[0]);
         int xi = 1;
@@ -691,7 +759,10 @@ gemv_kernel(const __grid_constant__ Batch<MAXI> p) {
     const uint32_t smem_s = smem_u32(smem);
     grid_dep_wait();                                     // x is written by the previous kernel
     if (i_first >= 0) {
-        stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, tid, kCoop);
+        if constexpr (FMT == kFmtW4G64)
+            stage_x_g64_wide<MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, tid, kCoop);
+        else
+            stage_x<FMT, MT>(p.it[i_first], p.m0, p.mrows, smem + p.x_off, tid, kCoop);
         asm volatile("bar.sync %0, %1;" :: "n"(kCoopBarrier), "n"(kCoop) : "memory");
     }
     Ring ring;

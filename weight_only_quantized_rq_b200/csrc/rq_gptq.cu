@@ -15,9 +15,15 @@
 // Cholesky and one triangular inverse. All of it runs in the caller's U
 // buffer:
 //   1. U := J (H + lambda I) J (dead diagonal entries set to 1 first);
-//   2. lower Cholesky in place, one launch per column (every warp recomputes
-//      the column's pivot from the row, so no launch writes what it reads);
-//      the diagonal is written by a last launch;
+//   2. lower Cholesky in place, in blocks of 32 columns: one CTA factors the
+//      32 x 32 diagonal block (the sums over the columns left of the block
+//      first, by all its warps, then the block's columns in order) and keeps
+//      each pivot in the strictly upper triangle (free until step 3); then
+//      one warp per row below the block forms the row's 32 entries (its sums
+//      over the left columns against the block's rows, staged 32 columns at
+//      a time in shared memory, then a forward solve with the block). Two
+//      launches per 32 columns instead of one per column; a last launch
+//      moves the pivots onto the diagonal;
 //   3. M^-1 by one forward substitution per column (a warp each), reading
 //      the lower triangle and writing column j of M^-1 transposed into row j
 //      of the strictly upper triangle, which no solve reads;
@@ -122,43 +128,131 @@ __global__ void __launch_bounds__(256) gptq_reverse_kernel(const double* __restr
         for (int k = threadIdx.x; k < K; k += 256) dead[k] = H[(size_t)k * K + k] == 0.0 ? 1 : 0;
 }
 
-// Pivot of column j from row j: sqrt(A[j][j] - sum_{p<j} L[j][p]^2), the same
-// operations in every caller (so every warp gets the same bits).
-__device__ __forceinline__ double chol_pivot(const double* A, int K, int j, int lane) {
-    const double* Lj = A + (size_t)j * K;
-    double s = 0.0;
-    for (int p = lane; p < j; p += 32) s = __fma_rn(Lj[p], Lj[p], s);
-    s = warp_sum(s);
-    const double d = A[(size_t)j * K + j] - s;
-    return d > 0.0 ? sqrt(d) : __longlong_as_double(0x7ff8000000000000ll);
+constexpr int kNB = 32;           // Cholesky block (columns)
+constexpr int kCh = 128;          // left columns staged per round
+constexpr int kDiagThreads = 1024;
+
+// A pivot that is not positive: NaN, and the status bit (no fault).
+__device__ __forceinline__ double chol_root(double d) {
+    if (d > 0.0) return sqrt(d);
+    atomicOr(&g_status, kStatusNotSpd);
+    return __longlong_as_double(0x7ff8000000000000ll);
 }
 
-// Step 2: column j of the lower Cholesky factor below the diagonal; warp w of
-// block b handles row i = j + 1 + 8 b + w.
-__global__ void __launch_bounds__(kWarps * 32) chol_col_kernel(double* __restrict__ A, int K, int j) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i = j + 1 + blockIdx.x * kWarps + warp;
-    if (i >= K) return;
-    const double ljj = chol_pivot(A, K, j, lane);
-    const double* Li = A + (size_t)i * K;
-    const double* Lj = A + (size_t)j * K;
-    double s = 0.0;
-    for (int p = lane; p < j; p += 32) s = __fma_rn(Li[p], Lj[p], s);
-    s = warp_sum(s);
-    if (lane == 0) A[(size_t)i * K + j] = (A[(size_t)i * K + j] - s) / ljj;
-}
-
-// Step 2, last launch: every diagonal entry from its (final) row.
-__global__ void __launch_bounds__(kWarps * 32) chol_diag_kernel(double* __restrict__ A, int K) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j = blockIdx.x * kWarps + warp;
-    if (j >= K) return;
-    const double ljj = chol_pivot(A, K, j, lane);
-    __syncwarp();
-    if (lane == 0) {
-        if (!(ljj > 0.0)) atomicOr(&g_status, kStatusNotSpd);
-        A[(size_t)j * K + j] = ljj;
+// Step 2a: the diagonal block [j0, j0 + nb) of the lower Cholesky factor (one
+// CTA). G[r][c] (r >= c) = sum over p < j0 of L[j0+r][p] L[j0+c][p], thread
+// (r, c) over the block's rows staged kCh columns at a time (in p order);
+// then column by column: the pivot d_c from row c, and rows r > c of column
+// c. G's lower part is overwritten by the block's L entries as they are
+// formed. Writes the block's strictly lower entries into A, and d_c into
+// A[j0+c][j0+c+1] (the strictly upper triangle is not read before step 3
+// overwrites it), or onto the diagonal for the last row of A.
+__global__ void __launch_bounds__(kDiagThreads) chol_block_diag_kernel(double* __restrict__ A, int K, int j0, int nb) {
+    __shared__ double T[kNB][kCh + 1];
+    __shared__ double G[kNB][kNB + 1];
+    __shared__ double piv;
+    const int tr = (int)threadIdx.x >> 5, tc = (int)threadIdx.x & 31;
+    double g = 0.0;
+    for (int p0 = 0; p0 < j0; p0 += kCh) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < nb * kCh; e += kDiagThreads) {
+            const int rr = e / kCh, l = e - rr * kCh;
+            T[rr][l] = p0 + l < j0 ? A[(size_t)(j0 + rr) * K + p0 + l] : 0.0;
+        }
+        __syncthreads();
+        if (tr < nb && tc <= tr)
+            for (int l = 0; l < kCh; ++l) g = __fma_rn(T[tr][l], T[tc][l], g);
     }
+    if (tr < nb && tc <= tr) G[tr][tc] = g;
+    __syncthreads();
+    for (int c = 0; c < nb; ++c) {
+        if (threadIdx.x == 0) {
+            double s = G[c][c];
+            for (int q = 0; q < c; ++q) s = __fma_rn(G[c][q], G[c][q], s);
+            const double d = chol_root(A[(size_t)(j0 + c) * K + j0 + c] - s);
+            piv = d;
+            if (j0 + c < K - 1) A[(size_t)(j0 + c) * K + j0 + c + 1] = d;
+            else A[(size_t)(j0 + c) * K + j0 + c] = d;
+        }
+        __syncthreads();
+        const int r = c + 1 + (int)threadIdx.x;
+        if (r < nb) {
+            double s = G[r][c];
+            for (int q = 0; q < c; ++q) s = __fma_rn(G[r][q], G[c][q], s);
+            const double v = (A[(size_t)(j0 + r) * K + j0 + c] - s) / piv;
+            G[r][c] = v;
+            A[(size_t)(j0 + r) * K + j0 + c] = v;
+        }
+        __syncthreads();
+    }
+}
+
+// Step 2b: rows i >= j0 + nb of the block's columns, one warp per row: the
+// sums over p < j0 of L[i][p] L[j0+c][p] for all c at once (the block's rows
+// staged kCh columns at a time in shared memory; lane l takes p = l, l + 32,
+// ... in order), then the forward solve with the block's lower triangle and
+// pivots.
+__global__ void __launch_bounds__(kWarps * 32) chol_block_panel_kernel(double* __restrict__ A, int K, int j0, int nb) {
+    __shared__ double T[kNB][kCh + 1];                // T[c][l] = L[j0+c][p0+l]
+    __shared__ double D[kNB][kNB + 1];                // the block: strict lower L, pivots on the diagonal
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = j0 + nb + (int)blockIdx.x * kWarps + warp;
+    const bool act = i < K;
+    for (int e = threadIdx.x; e < nb * nb; e += kWarps * 32) {
+        const int r = e / nb, c = e - r * nb;
+        if (r > c) D[r][c] = A[(size_t)(j0 + r) * K + j0 + c];
+        else if (r == c) D[r][r] = A[(size_t)(j0 + r) * K + j0 + r + 1];   // j0 + r < K - 1 here
+    }
+    const double* Li = A + (size_t)(act ? i : j0) * K;
+    double acc[kNB];
+#pragma unroll
+    for (int c = 0; c < kNB; ++c) acc[c] = 0.0;
+    for (int p0 = 0; p0 < j0; p0 += kCh) {
+        double li[kCh / 32];
+#pragma unroll
+        for (int k = 0; k < kCh / 32; ++k) {
+            const int p = p0 + 32 * k + lane;
+            li[k] = act && p < j0 ? Li[p] : 0.0;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < nb * kCh; e += kWarps * 32) {
+            const int c = e / kCh, l = e - c * kCh;
+            T[c][l] = p0 + l < j0 ? A[(size_t)(j0 + c) * K + p0 + l] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kCh / 32; ++k)
+#pragma unroll
+            for (int c = 0; c < kNB; ++c)
+                if (c < nb) acc[c] = __fma_rn(li[k], T[c][32 * k + lane], acc[c]);
+    }
+    __syncthreads();                                   // D is complete (also when j0 == 0)
+    if (!act) return;
+#pragma unroll
+    for (int c = 0; c < kNB; ++c) acc[c] = warp_sum(acc[c]);
+    double lr[kNB];                                    // L[i][j0 + c], the same in every lane
+#pragma unroll
+    for (int c = 0; c < kNB; ++c) {
+        if (c < nb) {
+            double s = acc[c];
+#pragma unroll
+            for (int q = 0; q < c; ++q) s = __fma_rn(lr[q], D[c][q], s);
+            lr[c] = (Li[j0 + c] - s) / D[c][c];
+        }
+    }
+    if (lane < nb) {
+        double v = 0.0;
+#pragma unroll
+        for (int c = 0; c < kNB; ++c)
+            if (c == lane) v = lr[c];
+        A[(size_t)i * K + j0 + lane] = v;
+    }
+}
+
+// Step 2c: the pivots onto the diagonal (the last row's is there already).
+__global__ void chol_pivots_kernel(double* __restrict__ A, int K) {
+    const int j = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    if (j < K - 1) A[(size_t)j * K + j] = A[(size_t)j * K + j + 1];
 }
 
 // Step 3: column j of M^-1 by forward substitution (M x = e_j): x_j = 1/M_jj,
@@ -226,13 +320,18 @@ cudaError_t launch_hessian(const void* x, int R, int K, double* H, cudaStream_t 
 cudaError_t launch_gptq_prepare(const double* H, int K, double damp, double* U, uint8_t* dead, cudaStream_t st) {
     gptq_reverse_kernel<<<(unsigned)K, 256, 0, st>>>(H, K, damp, U, dead);
     cudaError_t e = cudaGetLastError();
-    for (int j = 0; j + 1 < K && e == cudaSuccess; ++j) {
-        const int rows = K - 1 - j;
-        chol_col_kernel<<<(unsigned)((rows + kWarps - 1) / kWarps), kWarps * 32, 0, st>>>(U, K, j);
+    for (int j0 = 0; j0 < K && e == cudaSuccess; j0 += kNB) {
+        const int nb = K - j0 < kNB ? K - j0 : kNB;
+        chol_block_diag_kernel<<<1, kDiagThreads, 0, st>>>(U, K, j0, nb);
         e = cudaGetLastError();
+        const int rows = K - j0 - nb;
+        if (e == cudaSuccess && rows > 0) {
+            chol_block_panel_kernel<<<(unsigned)((rows + kWarps - 1) / kWarps), kWarps * 32, 0, st>>>(U, K, j0, nb);
+            e = cudaGetLastError();
+        }
     }
     if (e != cudaSuccess) return e;
-    chol_diag_kernel<<<(unsigned)((K + kWarps - 1) / kWarps), kWarps * 32, 0, st>>>(U, K);
+    chol_pivots_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(U, K);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // forward substitutions: one column of K doubles in shared memory per warp; fewer warps per block
     // for wide K

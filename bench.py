@@ -672,8 +672,8 @@ def run_ours(args, w, M):
                 "hessian_ms": round(ms_h, 3), "hessian_fp64_TFLOP_s": round(2.0 * K_g * K_g * R_g / (ms_h * 1e-3) / 1e12, 2),
                 "prepare_ms": round(ms_p, 3), "pack_ms": round(ms_q, 3),
                 "pack_fp64_GFLOP_s": round(N_g * K_g * K_g / (ms_q * 1e-3) / 1e9, 1),
-                "kernels": "hessian_kernel; gptq_reverse/chol_col (one launch per column)/chol_diag/trinv/"
-                           "gptq_finish; gptq_sym_kernel",
+                "kernels": "hessian_kernel; gptq_reverse/chol_block_diag + chol_block_panel (per 32 columns)/"
+                           "chol_pivots/trinv/gptq_finish; gptq_sym_kernel",
                 "note": "offline calibration steps, measured for reference; not part of the decode step"}
         del xg, Wg, Hg, Ug, dg, outg, basis
     status = rq.rq_device_status(stream)

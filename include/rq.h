@@ -288,7 +288,8 @@ int rq_hessian_accum(const void *x, int R, int K, double *H, void *stream);
  *         workspace too; it must not overlap H.
  *   dead  device [K] bytes, out: 1 where H's diagonal entry was 0.
  * Computed as J inv(chol(J H' J)) J (J reverses the index order): one
- * Cholesky and one triangular inverse, one launch per column (K launches).
+ * Cholesky (two launches per block of 32 columns) and one triangular inverse
+ * (a warp per column).
  * A non-positive pivot sets bit 5 of the device status word (see
  * rq_device_status) and leaves NaNs in U. Limits: 1 <= K <= 16384. */
 int rq_gptq_prepare(const double *H, int K, double damp, double *U, unsigned char *dead, void *stream);
